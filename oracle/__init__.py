@@ -1,0 +1,105 @@
+"""fp64 CPU oracle for gpt-oss-style grouped-query attention with sinks.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+bench's CPU-baseline leg may import this package. It shares no code with the
+CUDA library: the arithmetic lives in ``gptoss_attn_oracle.c`` (plain loops,
+fp64), wrapped here with ctypes, and ``brute.py`` holds a second, literal
+pure-Python transcription used to pin it on tiny inputs.
+
+Functions take numpy arrays of exact input values (bf16 inputs converted to
+fp64 without rounding) and return fp64 results.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+NQ, NKV, D = 64, 8, 64
+ROPE_THETA = 150000.0
+SCALE = 0.125
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int64)
+        lib.oracle_rope_rows.argtypes = [dp, dp, ctypes.c_int64, dp]
+        lib.oracle_prefill.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, dp]
+        lib.oracle_prefill_rows.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ip, ctypes.c_int64, dp]
+        lib.oracle_decode.argtypes = [dp, dp, dp, dp, ip, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, dp]
+        _lib = lib
+    return _lib
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a, t=ctypes.c_double):
+    return a.ctypes.data_as(ctypes.POINTER(t))
+
+
+def rope(x, pos):
+    """Rotate head vectors ``x[..., 64]`` by positions ``pos`` (shape ``x.shape[:-1]``)."""
+    x = _f64(x)
+    p = _f64(np.broadcast_to(pos, x.shape[:-1]))
+    y = np.empty_like(x)
+    _load().oracle_rope_rows(_ptr(x), _ptr(p), x.size // D, _ptr(y))
+    return y
+
+
+def _norm_window(window, seqlen):
+    return int(window) if window is not None else 0
+
+
+def prefill(q, k, v, sinks, pos, window):
+    """Attention output ``[B, S, 64, 64]`` (fp64) for every query row.
+
+    q: [B, S, 64, 64]; k, v: [B, S, 8, 64]; sinks: [64]; pos: [B, S];
+    window <= 0 means full causal, W > 0 the W-key sliding window.
+    """
+    q, k, v, sinks, pos = _f64(q), _f64(k), _f64(v), _f64(sinks), _f64(pos)
+    B, S = q.shape[0], q.shape[1]
+    out = np.empty((B, S, NQ, D), dtype=np.float64)
+    _load().oracle_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(pos), B, S,
+                           _norm_window(window, S), _ptr(out))
+    return out
+
+
+def prefill_rows(q, k, v, sinks, pos, window, rows):
+    """Attention output ``[n, 64, 64]`` for the query rows ``rows`` = [(b, i), ...]."""
+    q, k, v, sinks, pos = _f64(q), _f64(k), _f64(v), _f64(sinks), _f64(pos)
+    B, S = q.shape[0], q.shape[1]
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 2))
+    out = np.empty((r.shape[0], NQ, D), dtype=np.float64)
+    _load().oracle_prefill_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(pos), B, S,
+                                _norm_window(window, S), _ptr(r, ctypes.c_int64), r.shape[0],
+                                _ptr(out))
+    return out
+
+
+def decode(q, kcache, vcache, sinks, lengths, window):
+    """One decode step, ``[B, 64, 64]`` fp64.
+
+    q: [B, 64, 64] un-rotated (rotated here at position len-1);
+    kcache, vcache: [B, max_len, 8, 64], kcache already rotated; lengths: [B].
+    """
+    q, kc, vc, sinks = _f64(q), _f64(kcache), _f64(vcache), _f64(sinks)
+    L = np.ascontiguousarray(np.asarray(lengths, dtype=np.int64))
+    B, max_len = kc.shape[0], kc.shape[1]
+    out = np.empty((B, NQ, D), dtype=np.float64)
+    _load().oracle_decode(_ptr(q), _ptr(kc), _ptr(vc), _ptr(sinks), _ptr(L, ctypes.c_int64), B,
+                          max_len, int(window), _ptr(out))
+    return out
