@@ -1,0 +1,237 @@
+"""gpt-oss-style grouped-query attention with sinks on B200 (sm_100a).
+
+Thin ctypes binding over ``libgptoss_attn.so`` (C ABI in
+``include/gptoss_attn.h``). This module only marshals arguments: every step
+of the attention runs in the library's CUDA kernels. PyTorch supplies device
+memory and streams. There is no CPU fallback: if the library or a CUDA
+device is missing, calls raise.
+
+Shapes (bf16 unless noted):
+    prefill: q [B, S, 64, 64], k/v [B, S, 8, 64], sinks fp32 [64],
+             pos int32 [B, S]  ->  out [B, S, 64, 64]
+    decode:  q [B, 64, 64] (un-rotated), kcache/vcache [B, L, 8, 64]
+             (keys rotated), sinks fp32 [64], lengths int32 [B] -> out [B, 64, 64]
+``window <= 0`` is full causal; ``window = W > 0`` the W-key sliding window.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["prefill", "decode", "decode_workspace_bytes", "check", "init", "rope_table",
+           "library_path", "GptossAttnError", "NUM_HEADS", "NUM_KV_HEADS", "HEAD_DIM",
+           "MAX_POSITION"]
+
+NUM_HEADS = 64
+NUM_KV_HEADS = 8
+HEAD_DIM = 64
+MAX_POSITION = 131072
+ABI_VERSION = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libgptoss_attn.so"
+_lib = None
+
+
+class GptossAttnError(RuntimeError):
+    """A non-zero status returned by the C library."""
+
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s failed: %s (status %d)" % (what, _status_string(status), status))
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise ImportError("%s is not built; run `python -m attention_gqa_b200.build`" % path)
+    lib = ctypes.CDLL(path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.gptoss_attn_abi_version.restype = i32
+    lib.gptoss_attn_status_string.argtypes = [i32]
+    lib.gptoss_attn_status_string.restype = ctypes.c_char_p
+    lib.gptoss_attn_init.restype = i32
+    lib.gptoss_attn_rope_table.argtypes = [ctypes.POINTER(vp)]
+    lib.gptoss_attn_rope_table.restype = i32
+    lib.gptoss_attn_prefill.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, vp]
+    lib.gptoss_attn_prefill.restype = i32
+    lib.gptoss_attn_decode_workspace_bytes.argtypes = [i32, i32, i32]
+    lib.gptoss_attn_decode_workspace_bytes.restype = sz
+    lib.gptoss_attn_decode.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, vp, sz, vp]
+    lib.gptoss_attn_decode.restype = i32
+    lib.gptoss_attn_check.argtypes = [vp]
+    lib.gptoss_attn_check.restype = i32
+    if lib.gptoss_attn_abi_version() != ABI_VERSION:
+        raise ImportError("%s has ABI %d, expected %d" % (path, lib.gptoss_attn_abi_version(),
+                                                          ABI_VERSION))
+    _lib = lib
+    return lib
+
+
+def _status_string(status: int) -> str:
+    try:
+        return _load().gptoss_attn_status_string(status).decode()
+    except Exception:
+        return "unknown"
+
+
+def _raise(status: int, what: str):
+    if status != 0:
+        raise GptossAttnError(status, what)
+
+
+def _stream_handle(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dev(t: torch.Tensor, dtype, name: str, device) -> torch.Tensor:
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return t
+
+
+def _target_device(*ts):
+    for t in ts:
+        if t.device.type == "cuda":
+            return t.device
+    if not torch.cuda.is_available():
+        raise RuntimeError("gptoss attention needs a CUDA device (sm_100a); none is available")
+    return torch.device("cuda", torch.cuda.current_device())
+
+
+def init() -> None:
+    """Build the current device's rotary table (allocates; call before graph capture)."""
+    _raise(_load().gptoss_attn_init(), "gptoss_attn_init")
+
+
+class _DevicePtr:
+    """Exposes a library-owned device buffer to torch through __cuda_array_interface__."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (ptr, False), "version": 3}
+
+
+def rope_table() -> torch.Tensor:
+    """A copy of the device rotary table, fp32 [131072, 32, 2] of (cos, sin)."""
+    p = ctypes.c_void_p()
+    _raise(_load().gptoss_attn_rope_table(ctypes.byref(p)), "gptoss_attn_rope_table")
+    view = torch.as_tensor(_DevicePtr(p.value, (MAX_POSITION, HEAD_DIM // 2, 2), "<f4"),
+                           device="cuda")
+    return view.clone()
+
+
+def prefill(q, k, v, sinks, pos, window: int = 0, out=None, stream=None) -> torch.Tensor:
+    """Causal grouped-query attention with sinks over whole sequences.
+
+    Host (CPU) tensors are copied to the current CUDA device first and the
+    result is copied back, so the call works end to end from host memory.
+    """
+    lib = _load()
+    host = q.device.type != "cuda"
+    device = _target_device(q, k, v)
+    if host:
+        with torch.cuda.device(device):
+            s = stream if stream is not None else torch.cuda.current_stream()
+            with torch.cuda.stream(s):
+                res = prefill(q.to(device, non_blocking=True), k.to(device, non_blocking=True),
+                              v.to(device, non_blocking=True),
+                              sinks.to(device, non_blocking=True),
+                              pos.to(device, non_blocking=True), window, None, s)
+                if out is None:
+                    out = torch.empty(res.shape, dtype=res.dtype, pin_memory=True)
+                out.copy_(res, non_blocking=True)
+            s.synchronize()
+        return out
+    q = _dev(q, torch.bfloat16, "q", device)
+    k = _dev(k, torch.bfloat16, "k", device)
+    v = _dev(v, torch.bfloat16, "v", device)
+    sinks = _dev(sinks, torch.float32, "sinks", device)
+    pos = _dev(pos, torch.int32, "pos", device)
+    if q.dim() != 4 or q.shape[2:] != (NUM_HEADS, HEAD_DIM):
+        raise ValueError("q must be [B, S, 64, 64], got %s" % (tuple(q.shape),))
+    B, S = q.shape[0], q.shape[1]
+    for name, t in (("k", k), ("v", v)):
+        if tuple(t.shape) != (B, S, NUM_KV_HEADS, HEAD_DIM):
+            raise ValueError("%s must be [B, S, 8, 64], got %s" % (name, tuple(t.shape)))
+    if tuple(sinks.shape) != (NUM_HEADS,):
+        raise ValueError("sinks must be [64]")
+    if tuple(pos.shape) != (B, S):
+        raise ValueError("pos must be [B, S]")
+    dev_out = out if (out is not None and out.device.type == "cuda") else torch.empty(
+        (B, S, NUM_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=device)
+    st = lib.gptoss_attn_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), sinks.data_ptr(),
+                                 pos.data_ptr(), int(window), dev_out.data_ptr(), B, S,
+                                 _stream_handle(stream))
+    _raise(st, "gptoss_attn_prefill")
+    return dev_out
+
+
+def decode_workspace_bytes(batch: int, max_len: int, window: int = 0) -> int:
+    return int(_load().gptoss_attn_decode_workspace_bytes(batch, max_len, int(window)))
+
+
+def decode(q, kcache, vcache, sinks, lengths, window: int = 0, out=None, workspace=None,
+           stream=None) -> torch.Tensor:
+    """One decode step against a rotated key cache; see the module docstring."""
+    lib = _load()
+    host = q.device.type != "cuda"
+    device = _target_device(q, kcache, vcache)
+    if host:
+        with torch.cuda.device(device):
+            s = stream if stream is not None else torch.cuda.current_stream()
+            with torch.cuda.stream(s):
+                res = decode(q.to(device, non_blocking=True),
+                             kcache.to(device, non_blocking=True),
+                             vcache.to(device, non_blocking=True),
+                             sinks.to(device, non_blocking=True),
+                             lengths.to(device, non_blocking=True), window, None, workspace, s)
+                if out is None:
+                    out = torch.empty(res.shape, dtype=res.dtype, pin_memory=True)
+                out.copy_(res, non_blocking=True)
+            s.synchronize()
+        return out
+    q = _dev(q, torch.bfloat16, "q", device)
+    kcache = _dev(kcache, torch.bfloat16, "kcache", device)
+    vcache = _dev(vcache, torch.bfloat16, "vcache", device)
+    sinks = _dev(sinks, torch.float32, "sinks", device)
+    lengths = _dev(lengths, torch.int32, "lengths", device)
+    if q.dim() != 3 or q.shape[1:] != (NUM_HEADS, HEAD_DIM):
+        raise ValueError("q must be [B, 64, 64]")
+    B = q.shape[0]
+    if kcache.dim() != 4 or kcache.shape[0] != B or kcache.shape[2:] != (NUM_KV_HEADS, HEAD_DIM):
+        raise ValueError("kcache must be [B, L, 8, 64]")
+    if vcache.shape != kcache.shape:
+        raise ValueError("vcache must match kcache")
+    L = kcache.shape[1]
+    need = decode_workspace_bytes(B, L, window)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    dev_out = out if (out is not None and out.device.type == "cuda") else torch.empty(
+        (B, NUM_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=device)
+    st = lib.gptoss_attn_decode(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
+                                sinks.data_ptr(), lengths.data_ptr(), int(window),
+                                dev_out.data_ptr(), B, L, workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(),
+                                _stream_handle(stream))
+    _raise(st, "gptoss_attn_decode")
+    return dev_out
+
+
+def check(stream=None) -> None:
+    """Synchronize and raise if a kernel reported a device-side error."""
+    _raise(_load().gptoss_attn_check(_stream_handle(stream)), "gptoss_attn_check")

@@ -1,0 +1,222 @@
+// C-ABI entry points of libgptoss_attn.so: argument validation, per-device
+// state (rotary table, error word), TMA tensor maps, kernel launches.
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/gptoss_attn.h"
+#include "internal.h"
+#include "tmap.h"
+
+namespace {
+
+using namespace gqa;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  int* err = nullptr;       // 4-byte error word
+  float2* rope = nullptr;   // [kMaxPosition][32]
+};
+
+std::mutex g_mutex;
+DeviceState g_state[kMaxDevices];
+
+int current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices)
+    return GPTOSS_ATTN_ERR_NO_DEVICE;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+      major != 10)
+    return GPTOSS_ATTN_ERR_NO_DEVICE;
+  return GPTOSS_ATTN_OK;
+}
+
+// Allocates the error word (and, when asked, builds the rotary table) once
+// per device. Runs on the legacy default stream and waits for completion.
+int ensure_state(int dev, bool need_rope) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& st = g_state[dev];
+  if (!st.err) {
+    int* e = nullptr;
+    if (cudaMalloc(&e, sizeof(int)) != cudaSuccess) return GPTOSS_ATTN_ERR_ALLOC;
+    if (cudaMemset(e, 0, sizeof(int)) != cudaSuccess) {
+      cudaFree(e);
+      return GPTOSS_ATTN_ERR_LAUNCH;
+    }
+    st.err = e;
+  }
+  if (need_rope && !st.rope) {
+    float2* t = nullptr;
+    if (cudaMalloc(&t, sizeof(float2) * kMaxPosition * kRopePairs) != cudaSuccess)
+      return GPTOSS_ATTN_ERR_ALLOC;
+    if (launch_rope_table(t, nullptr) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+      cudaFree(t);
+      return GPTOSS_ATTN_ERR_LAUNCH;
+    }
+    st.rope = t;
+  }
+  return GPTOSS_ATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int gptoss_attn_abi_version(void) { return GPTOSS_ATTN_ABI_VERSION; }
+
+const char* gptoss_attn_status_string(int status) {
+  switch (status) {
+    case GPTOSS_ATTN_OK: return "ok";
+    case GPTOSS_ATTN_ERR_NULL_PTR: return "a required pointer is NULL";
+    case GPTOSS_ATTN_ERR_BAD_SHAPE: return "batch, seqlen or max_len out of range";
+    case GPTOSS_ATTN_ERR_BAD_ALIGN: return "a tensor base pointer is not 16-byte aligned";
+    case GPTOSS_ATTN_ERR_SMALL_WORKSPACE: return "workspace smaller than required";
+    case GPTOSS_ATTN_ERR_NO_DEVICE: return "no current CUDA device, or it is not sm_100";
+    case GPTOSS_ATTN_ERR_LAUNCH: return "a CUDA call or kernel launch failed";
+    case GPTOSS_ATTN_ERR_TENSOR_MAP: return "the driver rejected a TMA tensor map";
+    case GPTOSS_ATTN_ERR_ALLOC: return "library-owned device memory could not be allocated";
+    case GPTOSS_ATTN_ERR_DEVICE_TIMEOUT: return "a kernel pipeline wait timed out";
+    case GPTOSS_ATTN_ERR_BAD_POSITION: return "a rotary position was outside [0, 131072)";
+    case GPTOSS_ATTN_ERR_BAD_LENGTH: return "a decode length was outside [0, max_len]";
+    default: return "unknown status";
+  }
+}
+
+int gptoss_attn_init(void) {
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st != GPTOSS_ATTN_OK) return st;
+  return ensure_state(dev, true);
+}
+
+int gptoss_attn_rope_table(const void** table) {
+  if (!table) return GPTOSS_ATTN_ERR_NULL_PTR;
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, true);
+  if (st != GPTOSS_ATTN_OK) return st;
+  *table = g_state[dev].rope;
+  return GPTOSS_ATTN_OK;
+}
+
+int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float* sinks,
+                        const int32_t* pos, int window, void* out, int batch, int seqlen,
+                        cudaStream_t stream) {
+  if (!q || !k || !v || !sinks || !pos || !out) return GPTOSS_ATTN_ERR_NULL_PTR;
+  if (batch < 1 || seqlen < 1 || seqlen > kMaxPosition || batch > 65535)
+    return GPTOSS_ATTN_ERR_BAD_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(sinks) & 3u) || (reinterpret_cast<uintptr_t>(pos) & 3u))
+    return GPTOSS_ATTN_ERR_BAD_ALIGN;
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, true);
+  if (st != GPTOSS_ATTN_OK) return st;
+
+  PrefillMaps maps;
+  const uint64_t S = static_cast<uint64_t>(seqlen), B = static_cast<uint64_t>(batch);
+  const uint64_t qdims[4] = {kHeadDim, kNumHeads, S, B};
+  const uint64_t qstr[3] = {kHeadDim * 2, kNumHeads * kHeadDim * 2, S * kNumHeads * kHeadDim * 2};
+  const uint32_t qbox[4] = {kHeadDim, kGroup, 16, 1};
+  const uint64_t kdims[4] = {kHeadDim, kNumKvHeads, S, B};
+  const uint64_t kstr[3] = {kHeadDim * 2, kNumKvHeads * kHeadDim * 2,
+                            S * kNumKvHeads * kHeadDim * 2};
+  const uint32_t kbox[4] = {kHeadDim, 1, 128, 1};
+  if (!make_tmap_bf16_4d(&maps.q, q, qdims, qstr, qbox) ||
+      !make_tmap_bf16_4d(&maps.o, out, qdims, qstr, qbox) ||
+      !make_tmap_bf16_4d(&maps.k, k, kdims, kstr, kbox) ||
+      !make_tmap_bf16_4d(&maps.v, v, kdims, kstr, kbox))
+    return GPTOSS_ATTN_ERR_TENSOR_MAP;
+
+  PrefillArgs args;
+  args.pos = pos;
+  args.sinks = sinks;
+  args.rope = g_state[dev].rope;
+  args.err = g_state[dev].err;
+  args.batch = batch;
+  args.seqlen = seqlen;
+  args.window = window > 0 ? window : 0;
+  args.n_qtiles = (seqlen + 31) / 32;
+  return launch_prefill(maps, args, stream) == cudaSuccess ? GPTOSS_ATTN_OK
+                                                           : GPTOSS_ATTN_ERR_LAUNCH;
+}
+
+size_t gptoss_attn_decode_workspace_bytes(int batch, int max_len, int window) {
+  if (batch < 1 || max_len < 1 || batch > 65535) return 0;
+  int nsplit = 0, chunk = 0;
+  decode_plan(batch, max_len, window, &nsplit, &chunk);
+  return decode_workspace_bytes(batch, nsplit);
+}
+
+int gptoss_attn_decode(const void* q, const void* kcache, const void* vcache, const float* sinks,
+                       const int32_t* len, int window, void* out, int batch, int max_len,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !kcache || !vcache || !sinks || !len || !out || !workspace)
+    return GPTOSS_ATTN_ERR_NULL_PTR;
+  if (batch < 1 || max_len < 1 || batch > 65535) return GPTOSS_ATTN_ERR_BAD_SHAPE;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(sinks) & 3u) ||
+      (reinterpret_cast<uintptr_t>(len) & 3u))
+    return GPTOSS_ATTN_ERR_BAD_ALIGN;
+  int nsplit = 0, chunk = 0;
+  decode_plan(batch, max_len, window, &nsplit, &chunk);
+  const size_t need = decode_workspace_bytes(batch, nsplit);
+  if (workspace_bytes < need) return GPTOSS_ATTN_ERR_SMALL_WORKSPACE;
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, false);
+  if (st != GPTOSS_ATTN_OK) return st;
+
+  DecodeMaps maps;
+  const uint64_t L = static_cast<uint64_t>(max_len), B = static_cast<uint64_t>(batch);
+  const uint64_t dims[4] = {kHeadDim, kNumKvHeads, L, B};
+  const uint64_t str[3] = {kHeadDim * 2, kNumKvHeads * kHeadDim * 2,
+                           L * kNumKvHeads * kHeadDim * 2};
+  const uint32_t box[4] = {kHeadDim, 1, 64, 1};
+  if (!make_tmap_bf16_4d(&maps.k, kcache, dims, str, box) ||
+      !make_tmap_bf16_4d(&maps.v, vcache, dims, str, box))
+    return GPTOSS_ATTN_ERR_TENSOR_MAP;
+
+  DecodeArgs a;
+  a.q = static_cast<const uint16_t*>(q);
+  a.kcache = static_cast<const uint16_t*>(kcache);
+  a.vcache = static_cast<const uint16_t*>(vcache);
+  a.sinks = sinks;
+  a.len = len;
+  a.out = static_cast<uint16_t*>(out);
+  const size_t rows = static_cast<size_t>(batch) * kNumHeads * nsplit;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + rows * kHeadDim * 4);
+  a.err = g_state[dev].err;
+  a.batch = batch;
+  a.max_len = max_len;
+  a.window = window > 0 ? window : 0;
+  a.nsplit = nsplit;
+  a.chunk = chunk;
+  return launch_decode(maps, a, stream) == cudaSuccess ? GPTOSS_ATTN_OK : GPTOSS_ATTN_ERR_LAUNCH;
+}
+
+int gptoss_attn_check(cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return GPTOSS_ATTN_ERR_NO_DEVICE;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return GPTOSS_ATTN_ERR_LAUNCH;
+  int* e = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    e = g_state[dev].err;
+  }
+  if (!e) return GPTOSS_ATTN_OK;
+  int h = 0;
+  if (cudaMemcpy(&h, e, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemset(e, 0, sizeof(int)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+    return GPTOSS_ATTN_ERR_LAUNCH;
+  if (h & kErrTimeout) return GPTOSS_ATTN_ERR_DEVICE_TIMEOUT;
+  if (h & kErrPosition) return GPTOSS_ATTN_ERR_BAD_POSITION;
+  if (h & kErrLength) return GPTOSS_ATTN_ERR_BAD_LENGTH;
+  return GPTOSS_ATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// Library-internal declarations shared by the host entry points and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace gqa {
+
+constexpr int kNumHeads = 64;
+constexpr int kNumKvHeads = 8;
+constexpr int kGroup = kNumHeads / kNumKvHeads;  // query heads per key/value head
+constexpr int kHeadDim = 64;
+constexpr int kRopePairs = kHeadDim / 2;
+constexpr int kMaxPosition = 131072;
+constexpr double kRopeTheta = 150000.0;
+
+// Device error word bits (set by kernels, read by gptoss_attn_check). After a
+// timeout the kernels skip their work until the word is cleared.
+constexpr int kErrTimeout = 1;
+constexpr int kErrPosition = 2;
+constexpr int kErrLength = 4;
+
+// Pipeline waits give up after this long (a healthy wait lasts microseconds).
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+
+struct PrefillArgs {
+  const int32_t* pos;   // [B][S]
+  const float* sinks;   // [64]
+  const float2* rope;   // [kMaxPosition][32] (cos, sin)
+  int* err;             // device error word
+  int batch;
+  int seqlen;
+  int window;           // <= 0: full causal
+  int n_qtiles;         // ceil(seqlen / 32)
+};
+
+struct PrefillMaps {
+  CUtensorMap q, k, v, o;
+};
+
+// Launches the prefill kernel; returns a cudaError_t.
+cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream);
+
+// Fills the rotary table [kMaxPosition][32] of (cos, sin).
+cudaError_t launch_rope_table(float2* table, cudaStream_t stream);
+
+struct DecodeArgs {
+  const uint16_t* q;       // [B][64][64] bf16, un-rotated
+  const uint16_t* kcache;  // [B][L][8][64] bf16
+  const uint16_t* vcache;  // [B][L][8][64] bf16
+  const float* sinks;      // [64]
+  const int32_t* len;      // [B]
+  uint16_t* out;           // [B][64][64] bf16
+  float* part_o;           // [B][64][nsplit][64]
+  float2* part_ml;         // [B][64][nsplit] (max in log2 units, sum)
+  int* err;
+  int batch;
+  int max_len;
+  int window;
+  int nsplit;
+  int chunk;               // keys per split
+};
+
+struct DecodeMaps {
+  CUtensorMap k, v;
+};
+
+cudaError_t launch_decode(const DecodeMaps& maps, const DecodeArgs& args, cudaStream_t stream);
+
+// Decode split planning shared by the workspace query and the launch.
+void decode_plan(int batch, int max_len, int window, int* nsplit, int* chunk);
+size_t decode_workspace_bytes(int batch, int nsplit);
+
+}  // namespace gqa

@@ -1,0 +1,412 @@
+"""Throughput of the gpt-oss attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole path over one batch of synthetic inputs:
+  * prefill, B=1, S=4096, 64 query / 8 key-value heads, head_dim 64: a
+    128-token sliding-window layer, then a full-causal layer, each with its
+    own seeded q/k/v/sinks (RoPE table, rotation, QK^T, sink-seeded online
+    softmax, PV, epilogue);
+  * decode, B=64 sequences against a bf16 cache of 8192 tokens: one
+    full-causal layer and one sliding layer (its last 128 entries)
+    (split-KV partials + log-sum-exp combine).
+``value`` is the prefill attention throughput in TFLOP/s counting unmasked
+FLOPs only (4 * 64 * 64 per visible (query, key) pair per head); the decode
+half of the metric (HBM GB/s over the algorithmic bytes) is reported in the
+``decode`` object. L2 is flushed (256 MB write) before every step, outside
+the timed events. Per-kernel times come from CUDA events on the launching
+stream. With N > 1 (torchrun), every rank runs the same per-GPU workload
+(weak scaling, no collective on the data path); times are the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "attention TFLOP/s (unmasked) & % bf16 peak; decode HBM GB/s & % of peak"
+NQ, NKV, D = 64, 8, 64
+PREFILL_B, PREFILL_S = 1, 4096
+PREFILL_LAYERS = ((0, 128), (1, 0))          # (layer index, window): sliding then full
+DECODE_B, DECODE_L = 64, 8192
+DECODE_LAYERS = ((0, 0), (1, 128))            # full, then sliding
+WORKLOAD = ("prefill B=1 S=4096 64q/8kv d64 (W=128 layer + full-causal layer) + "
+            "decode B=64 L=8192 (full layer + W=128 layer)")
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "prefill_full_S4096_traffic.txt")
+
+
+def visible_pairs(S: int, window: int) -> int:
+    if window <= 0 or window >= S:
+        return S * (S + 1) // 2
+    return window * S - window * (window - 1) // 2
+
+
+def prefill_flops(B: int, S: int, window: int) -> float:
+    return 4.0 * D * NQ * B * visible_pairs(S, window)
+
+
+def prefill_bytes(B: int, S: int) -> float:
+    return float(B * S * (2 * NQ * D * 2 + 2 * NKV * D * 2))  # q, out, k, v (bf16)
+
+
+def decode_bytes(B: int, L: int, window: int) -> float:
+    n = L if window <= 0 else min(window, L)
+    return float(B * n * NKV * D * 2 * 2 + 2 * B * NQ * D * 2)  # visible K and V, q, out
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), \
+            "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def source_digest() -> str:
+    p = os.path.join(ROOT, "attention_gqa_b200", "csrc", "prefill_sm100.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the full-causal prefill kernel from the committed
+    ncu summary, if it was taken on the current kernel source."""
+    try:
+        vals = {}
+        with open(PROFILE_TRAFFIC) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    vals[k.strip()] = v.strip()
+        if vals.get("kernel_source_sha256_16") != source_digest():
+            return None
+        return float(vals["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clocks and clock-event reasons through NVML while timing runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+
+def oracle_sample(budget_s: float = 12.0):
+    """Times the fp64 oracle on evenly spaced query rows of the two prefill
+    layers (all 64 heads of each row); returns (TFLOP/s, seconds, rows, FLOPs)."""
+    import oracle
+    import synth
+    oracle._load()
+    total_flops, total_s, nrows = 0.0, 0.0, 0
+    per_layer = budget_s / len(PREFILL_LAYERS)
+    for layer, window in PREFILL_LAYERS:
+        x = synth.make_prefill_inputs(2, layer, PREFILL_B, PREFILL_S)
+        k = synth.bf16_bits_to_f64(x["k"])
+        v = synth.bf16_bits_to_f64(x["v"])
+        n = 64
+        while True:
+            toks = np.linspace(0, PREFILL_S - 1, n).astype(np.int64)
+            rows = [(0, int(t)) for t in toks]
+            q_rows = synth.bf16_bits_to_f64(np.stack([x["q"][0, t] for t in toks]))
+            t0 = time.perf_counter()
+            oracle.prefill_rows(q_rows, k, v, x["sinks"], x["pos"], window, rows)
+            dt = time.perf_counter() - t0
+            if dt >= per_layer / 3 or n >= PREFILL_S:
+                break
+            n = min(PREFILL_S, n * 4)
+        flops = sum(4.0 * D * NQ * (min(t + 1, window) if window > 0 else t + 1) for t in toks)
+        total_flops += flops
+        total_s += dt
+        nrows += n
+    return total_flops / total_s / 1e12, total_s, nrows, total_flops
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return 0
+    value, secs, nrows, flops = oracle_sample()
+    cores = host_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": "%d evenly spaced query rows (all 64 heads) of the two prefill "
+                                   "layers, %.3g unmasked FLOPs" % (nrows, flops)},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU leg
+
+def run_ours(args, rank: int, world: int):
+    import torch
+    import torch.distributed as dist
+
+    import attention_gqa_b200 as gqa
+    import synth
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+    if rank == 0:
+        from attention_gqa_b200 import build
+        build.build()
+    if world > 1:
+        dist.barrier()
+    gqa.init()
+    stream = torch.cuda.current_stream()
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    # inputs resident in HBM
+    pre = []
+    for layer, window in PREFILL_LAYERS:
+        x = synth.make_prefill_inputs(2, layer, PREFILL_B, PREFILL_S)
+        pre.append(dict(q=to_dev(x["q"]), k=to_dev(x["k"]), v=to_dev(x["v"]),
+                        sinks=torch.from_numpy(x["sinks"]).to(dev),
+                        pos=torch.from_numpy(x["pos"]).to(dev), window=window,
+                        out=torch.empty(PREFILL_B, PREFILL_S, NQ, D, dtype=torch.bfloat16,
+                                        device=dev), host=x))
+    dec = []
+    for layer, window in DECODE_LAYERS:
+        x = synth.make_decode_inputs(4, layer, DECODE_B, DECODE_L)
+        ws = torch.empty(gqa.decode_workspace_bytes(DECODE_B, DECODE_L, window),
+                         dtype=torch.uint8, device=dev)
+        dec.append(dict(q=to_dev(x["q"]), kc=to_dev(x["kcache"]), vc=to_dev(x["vcache"]),
+                        sinks=torch.from_numpy(x["sinks"]).to(dev),
+                        len=torch.from_numpy(x["len"]).to(dev), window=window, ws=ws,
+                        out=torch.empty(DECODE_B, NQ, D, dtype=torch.bfloat16, device=dev)))
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        i = 0
+        if ev is not None:
+            ev[i].record(stream)
+        for p in pre:
+            gqa.prefill(p["q"], p["k"], p["v"], p["sinks"], p["pos"], p["window"], out=p["out"])
+            i += 1
+            if ev is not None:
+                ev[i].record(stream)
+        for d in dec:
+            gqa.decode(d["q"], d["kc"], d["vc"], d["sinks"], d["len"], d["window"], out=d["out"],
+                       workspace=d["ws"])
+            i += 1
+            if ev is not None:
+                ev[i].record(stream)
+
+    n_marks = 1 + len(PREFILL_LAYERS) + len(DECODE_LAYERS)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    gqa.check()
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks)]
+              for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_wall = time.perf_counter()
+        for s in range(args.steps):
+            flush.fill_(s & 0xFF)
+            step(events[s])
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        dist.barrier()
+    gqa.check()
+
+    seg = np.array([[events[s][i].elapsed_time(events[s][i + 1]) for i in range(n_marks - 1)]
+                    for s in range(args.steps)])  # ms, [steps, kernels]
+    seg_total = seg.sum(axis=0)                                       # ms per segment over K steps
+    if world > 1:
+        t = torch.tensor(seg_total, dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        seg_total = t.cpu().numpy()
+    npre = len(PREFILL_LAYERS)
+    pre_ms = float(seg_total[:npre].sum()) / args.steps
+    dec_ms = float(seg_total[npre:].sum()) / args.steps
+    step_ms = pre_ms + dec_ms
+    pre_flops = sum(prefill_flops(PREFILL_B, PREFILL_S, w) for _, w in PREFILL_LAYERS)
+    dec_bytes = sum(decode_bytes(DECODE_B, DECODE_L, w) for _, w in DECODE_LAYERS)
+    value = world * pre_flops / (pre_ms * 1e-3) / 1e12
+    dec_gbs = world * dec_bytes / (dec_ms * 1e-3) / 1e9
+
+    hbm, tf_burst, tf_sus, peak_src = load_peaks()
+    # dominant kernel: the full-causal prefill layer
+    full_idx = [i for i, (_, w) in enumerate(PREFILL_LAYERS) if w <= 0][0]
+    full_ms = float(seg_total[full_idx]) / args.steps
+    full_tf = prefill_flops(PREFILL_B, PREFILL_S, 0) / (full_ms * 1e-3) / 1e12
+    dfull_idx = npre + [i for i, (_, w) in enumerate(DECODE_LAYERS) if w <= 0][0]
+    dfull_ms = float(seg_total[dfull_idx]) / args.steps
+    dfull_gbs = decode_bytes(DECODE_B, DECODE_L, 0) / (dfull_ms * 1e-3) / 1e9
+
+    # end to end through the public API from pinned host buffers (prefill layers)
+    def pinned(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+            torch.bfloat16).pin_memory()
+    hostin = []
+    h2d = d2h = 0
+    for p in pre:
+        x = p["host"]
+        hq, hk, hv = pinned(x["q"]), pinned(x["k"]), pinned(x["v"])
+        hs, hp = torch.from_numpy(x["sinks"]).pin_memory(), torch.from_numpy(x["pos"]).pin_memory()
+        ho = torch.empty(p["out"].shape, dtype=torch.bfloat16).pin_memory()
+        hostin.append((hq, hk, hv, hs, hp, p["window"], ho))
+        h2d += sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs, hp))
+        d2h += ho.numel() * ho.element_size()
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        for hq, hk, hv, hs, hp, w, ho in hostin:
+            gqa.prefill(hq, hk, hv, hs, hp, w, out=ho)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for hq, hk, hv, hs, hp, w, ho in hostin:
+            gqa.prefill(hq, hk, hv, hs, hp, w, out=ho)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * pre_flops / (e2e_ms * 1e-3) / 1e12
+
+    if rank == 0:
+        cpu = None
+        if world == 1:
+            v, secs, nrows, flops = oracle_sample()
+            cpu = {"value": v, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+                   "sample": "%d evenly spaced query rows (all 64 heads) of the two prefill "
+                             "layers, %.3g unmasked FLOPs, %.1f s" % (nrows, flops, secs)}
+        traffic = profiled_traffic()
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) bf16 q/k/v and caches, N(0,1) fp32 sinks",
+            "config": {"workload": WORKLOAD, "l2": "flushed before every step (256 MB write)",
+                       "parallelism": "dp%d (independent replicas)" % world,
+                       "prefill_ms_per_step": pre_ms, "decode_ms_per_step": dec_ms,
+                       "wall_s": t_wall},
+            "roofline": {"kernel": "prefill_kernel (full-causal layer, S=4096)", "bound": "tensor",
+                         "achieved": full_tf, "peak": tf_burst, "unit": "TFLOP/s",
+                         "frac": full_tf / tf_burst, "peak_source": peak_src + " (burst)",
+                         "traffic": traffic,
+                         "algorithmic_bytes": prefill_bytes(PREFILL_B, PREFILL_S),
+                         "launch_ms": full_ms},
+            "decode": {"value": dec_gbs, "unit": "GB/s", "frac": dec_gbs / world / hbm,
+                       "peak": hbm, "full_layer_gbs": dfull_gbs,
+                       "full_layer_frac": dfull_gbs / hbm, "full_layer_ms": dfull_ms},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "what": "prefill layers via host buffers"},
+            "gpu_launches": args.steps * (len(PREFILL_LAYERS) + 2 * len(DECODE_LAYERS)),
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    return run_ours(args, rank, world)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,153 @@
+/*
+ * gptoss_attn — gpt-oss-style causal grouped-query attention with learned
+ * sinks, for NVIDIA B200 (sm_100a). C ABI of libgptoss_attn.so.
+ *
+ * The operation (gpt-oss pages):
+ *   - 64 query heads share 8 key/value heads; query head h reads key/value
+ *     head floor(h / 8) (inteligile "gpt-oss-120b" techniques map, row
+ *     "Grouped-query attention"; llm-atlas gpt-oss-20b field table:
+ *     num_attention_heads 64, num_key_value_heads 8, head_dim 64).
+ *   - queries and keys are rotated by the half-split rotary embedding,
+ *     theta = 150000, pair k = (element k, element k+32) turning by
+ *     pos * theta^(-2k/64) (techniques map rows "Partial RoPE" and
+ *     "Layers without positional encoding (NoPE)"; rope_theta in the
+ *     llm-atlas field table).
+ *   - scores are scaled by 1/sqrt(64); a per-head learned sink logit
+ *     sigma_h (unscaled) joins the softmax denominator and carries no value
+ *     (techniques map row "Learnable attention sink").
+ *   - full-causal layers, or sliding-window causal layers in which query i
+ *     sees keys i-W < j <= i (W = 128 in the model; techniques map rows
+ *     "Sliding-window attention", "Interleaved sliding-window and global
+ *     attention"; sliding_window in the llm-atlas field tables).
+ *
+ *   out[b,i,h,:] = sum_j p_j v[b,j,h/8,:],
+ *   p_j = exp(s_j) / (exp(sigma_h) + sum_j' exp(s_j')),
+ *   s_j = (R(pos_i) q[b,i,h]) . (R(pos_j) k[b,j,h/8]) / 8.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are bf16 (raw 16-bit patterns), row-major, contiguous,
+ *     device memory owned by the caller. The library keeps no pointer
+ *     after a call returns. Base pointers must be 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream).
+ *   - The return value is GPTOSS_ATTN_OK (0) or a negative status code;
+ *     no call aborts or prints. Argument errors are reported before any
+ *     work is enqueued. Faults detected inside a kernel set a device error
+ *     word that gptoss_attn_check() reports and clears.
+ *   - Accumulation is fp32; the rotated q/k and the probabilities are
+ *     rounded to bf16 for the tensor-core products; the output is rounded
+ *     to bf16 once.
+ */
+#ifndef GPTOSS_ATTN_H
+#define GPTOSS_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cudaStream_t;
+
+#define GPTOSS_ATTN_ABI_VERSION 1
+
+#define GPTOSS_ATTN_NUM_HEADS 64
+#define GPTOSS_ATTN_NUM_KV_HEADS 8
+#define GPTOSS_ATTN_HEAD_DIM 64
+#define GPTOSS_ATTN_MAX_POSITION 131072
+
+enum gptoss_attn_status {
+  GPTOSS_ATTN_OK = 0,
+  GPTOSS_ATTN_ERR_NULL_PTR = -1,        /* a required pointer is NULL */
+  GPTOSS_ATTN_ERR_BAD_SHAPE = -2,       /* batch, seqlen or max_len out of range */
+  GPTOSS_ATTN_ERR_BAD_ALIGN = -3,       /* a tensor base pointer is not 16-byte aligned */
+  GPTOSS_ATTN_ERR_SMALL_WORKSPACE = -4, /* workspace smaller than required */
+  GPTOSS_ATTN_ERR_NO_DEVICE = -5,       /* no current device, or it is not sm_100 */
+  GPTOSS_ATTN_ERR_LAUNCH = -6,          /* a CUDA call or kernel launch failed */
+  GPTOSS_ATTN_ERR_TENSOR_MAP = -7,      /* the driver rejected a TMA tensor map */
+  GPTOSS_ATTN_ERR_ALLOC = -8,           /* library-owned device memory could not be allocated */
+  GPTOSS_ATTN_ERR_DEVICE_TIMEOUT = -9,  /* a kernel pipeline wait ran out (reported by check) */
+  GPTOSS_ATTN_ERR_BAD_POSITION = -10,   /* a position was outside [0, 131072) (reported by check) */
+  GPTOSS_ATTN_ERR_BAD_LENGTH = -11      /* a decode length was outside [0, max_len] (reported by check) */
+};
+
+/* ABI version of the loaded library (GPTOSS_ATTN_ABI_VERSION). */
+int gptoss_attn_abi_version(void);
+
+/* Static description of a status code; never NULL. */
+const char* gptoss_attn_status_string(int status);
+
+/*
+ * Prepares the current device: builds the library-owned rotary table
+ * (cos, sin of pos * theta^(-2k/64) for every pos < 131072 and k < 32,
+ * evaluated in fp64 and stored as fp32, 33.5 MB) and a 4-byte device error
+ * word. Idempotent and thread-safe. gptoss_attn_prefill() calls it on its
+ * first use on a device; call it explicitly before capturing a CUDA graph,
+ * since it allocates. The memory is released when the process exits.
+ */
+int gptoss_attn_init(void);
+
+/*
+ * Diagnostics: stores in *table the device address of the current device's
+ * rotary table, fp32 pairs (cos, sin) laid out [131072][32], building it
+ * first if needed. The table is read-only and owned by the library.
+ */
+int gptoss_attn_rope_table(const void** table);
+
+/*
+ * Prefill: causal grouped-query attention over whole sequences.
+ *   q      bf16 [batch][seqlen][64][64]   (token-major, as the projections emit)
+ *   k, v   bf16 [batch][seqlen][8][64]
+ *   sinks  fp32 [64] (device), the per-head sink logits sigma_h; -inf allowed
+ *   pos    int32 [batch][seqlen] (device), rotary positions in [0, 131072);
+ *          masking uses token indices, positions only drive the rotation
+ *   window <= 0: full causal; W > 0: key j visible to query i iff i-W < j <= i
+ *   out    bf16 [batch][seqlen][64][64]; must not overlap the inputs
+ *   batch >= 1, 1 <= seqlen <= 131072 (batch * seqlen * 8 KB must fit the device)
+ * q and k are rotated inside the kernel; k and v are read as given.
+ */
+int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float* sinks,
+                        const int32_t* pos, int window, void* out, int batch, int seqlen,
+                        cudaStream_t stream);
+
+/*
+ * Bytes of device workspace gptoss_attn_decode() needs for these sizes.
+ * Returns 0 for invalid sizes.
+ */
+size_t gptoss_attn_decode_workspace_bytes(int batch, int max_len, int window);
+
+/*
+ * Decode: one new query token per sequence against a key/value cache.
+ *   q       bf16 [batch][64][64], not yet rotated; it is rotated here at
+ *           position len[b]-1
+ *   kcache  bf16 [batch][max_len][8][64], keys already rotated at their positions
+ *   vcache  bf16 [batch][max_len][8][64]
+ *   sinks   fp32 [64] (device)
+ *   len     int32 [batch] (device), the number of cached tokens, the new one
+ *           included; 0 <= len[b] <= max_len (len 0 gives a zero output)
+ *   window  <= 0: keys [0, len); W > 0: keys [max(0, len-W), len)
+ *   out     bf16 [batch][64][64]
+ *   workspace, workspace_bytes: caller-owned device scratch of at least
+ *           gptoss_attn_decode_workspace_bytes(batch, max_len, window) bytes,
+ *           16-byte aligned; its contents need no initialisation and are
+ *           garbage afterwards. Calls that overlap in time need separate
+ *           workspaces.
+ */
+int gptoss_attn_decode(const void* q, const void* kcache, const void* vcache, const float* sinks,
+                       const int32_t* len, int window, void* out, int batch, int max_len,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears the current device's error
+ * word. Returns GPTOSS_ATTN_OK, GPTOSS_ATTN_ERR_DEVICE_TIMEOUT,
+ * GPTOSS_ATTN_ERR_BAD_POSITION, GPTOSS_ATTN_ERR_BAD_LENGTH or
+ * GPTOSS_ATTN_ERR_LAUNCH (a CUDA error surfaced by the synchronization).
+ * While the error word is set, kernels skip their work.
+ */
+int gptoss_attn_check(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTOSS_ATTN_H */

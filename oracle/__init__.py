@@ -78,11 +78,16 @@ def prefill(q, k, v, sinks, pos, window):
     return out
 
 
-def prefill_rows(q, k, v, sinks, pos, window, rows):
-    """Attention output ``[n, 64, 64]`` for the query rows ``rows`` = [(b, i), ...]."""
-    q, k, v, sinks, pos = _f64(q), _f64(k), _f64(v), _f64(sinks), _f64(pos)
-    B, S = q.shape[0], q.shape[1]
+def prefill_rows(q_rows, k, v, sinks, pos, window, rows):
+    """Attention output ``[n, 64, 64]`` for the query rows ``rows`` = [(b, i), ...].
+
+    ``q_rows[n]`` is the query vector block ``[64, 64]`` of row ``rows[n]``;
+    k, v: [B, S, 8, 64]; pos: [B, S].
+    """
+    q, k, v, sinks, pos = _f64(q_rows), _f64(k), _f64(v), _f64(sinks), _f64(pos)
+    B, S = k.shape[0], k.shape[1]
     r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 2))
+    assert q.shape == (r.shape[0], NQ, D)
     out = np.empty((r.shape[0], NQ, D), dtype=np.float64)
     _load().oracle_prefill_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(pos), B, S,
                                 _norm_window(window, S), _ptr(r, ctypes.c_int64), r.shape[0],

@@ -103,12 +103,13 @@ static void attend_row(const double* qr, const double* kr, const double* v, int6
 
 /*
  * Prefill oracle on selected query rows.
- *   q    [B][S][64][64], k, v [B][S][8][64], sinks [64], pos [B][S] (fp64 values)
+ *   q_rows [nrows][64][64]: the query vectors of the selected rows
+ *   k, v [B][S][8][64], sinks [64], pos [B][S] (fp64 values)
  *   window: <= 0 full causal, else W
  *   rows: nrows pairs (b, i) of query rows to compute; out [nrows][64][64]
  * Every head of each selected row is computed.
  */
-void oracle_prefill_rows(const double* q, const double* k, const double* v, const double* sinks,
+void oracle_prefill_rows(const double* q_rows, const double* k, const double* v, const double* sinks,
                          const double* pos, int B, int S, int window, const int64_t* rows,
                          int64_t nrows, double* out) {
   double* kr = (double*)malloc((size_t)S * D * sizeof(double));
@@ -133,7 +134,7 @@ void oracle_prefill_rows(const double* q, const double* k, const double* v, cons
           int64_t lo = window > 0 ? (i - window + 1 > 0 ? i - window + 1 : 0) : 0;
           for (int hh = 0; hh < GROUP; ++hh) {
             int h = g * GROUP + hh;
-            oracle_rope(q + (((int64_t)b * S + i) * NQ + h) * D, pos[(int64_t)b * S + i], qr);
+            oracle_rope(q_rows + (r * NQ + h) * D, pos[(int64_t)b * S + i], qr);
             attend_row(qr, kr, vg, (int64_t)NKV * D, lo, i, sinks[h], s, out + (r * NQ + h) * D);
           }
         }
@@ -144,7 +145,8 @@ void oracle_prefill_rows(const double* q, const double* k, const double* v, cons
   free(kr);
 }
 
-/* Prefill oracle on every query row: out [B][S][64][64]. */
+/* Prefill oracle on every query row: out [B][S][64][64]. Row r = b*S + i of q
+ * is query row (b, i), so q serves directly as the row list. */
 void oracle_prefill(const double* q, const double* k, const double* v, const double* sinks,
                     const double* pos, int B, int S, int window, double* out) {
   int64_t n = (int64_t)B * S;

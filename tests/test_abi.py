@@ -1,0 +1,106 @@
+"""The C-ABI library loads, exports every symbol the header declares, and
+rejects bad arguments on the host before any CUDA work (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import attention_gqa_b200 as gqa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gptoss_attn.h")
+
+
+def _header_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(gptoss_attn_\w+)\s*\(", text)))
+
+
+def _header_codes():
+    text = open(HEADER).read()
+    return {m.group(1): int(m.group(2))
+            for m in re.finditer(r"(GPTOSS_ATTN_(?:OK|ERR_\w+))\s*=\s*(-?\d+)", text)}
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from attention_gqa_b200 import build
+    build.build()
+    return gqa._load()
+
+
+def test_exports_every_declared_symbol(lib):
+    syms = _header_symbols()
+    assert len(syms) >= 8
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.gptoss_attn_abi_version() == 1
+    codes = _header_codes()
+    assert codes["GPTOSS_ATTN_OK"] == 0
+    strings = set()
+    for name, code in codes.items():
+        s = lib.gptoss_attn_status_string(code).decode()
+        assert s and s != "unknown status", name
+        strings.add(s)
+    assert len(strings) == len(codes)
+    assert lib.gptoss_attn_status_string(12345).decode() == "unknown status"
+
+
+def _prefill(lib, q=16, k=32, v=48, sinks=64, pos=80, window=0, out=96, batch=1, seqlen=8):
+    return lib.gptoss_attn_prefill(q, k, v, sinks, pos, window, out, batch, seqlen, None)
+
+
+def test_prefill_argument_errors(lib):
+    c = _header_codes()
+    assert _prefill(lib, q=None) == c["GPTOSS_ATTN_ERR_NULL_PTR"]
+    assert _prefill(lib, out=None) == c["GPTOSS_ATTN_ERR_NULL_PTR"]
+    assert _prefill(lib, batch=0) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert _prefill(lib, seqlen=0) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert _prefill(lib, seqlen=131073) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert _prefill(lib, k=40) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
+    assert _prefill(lib, pos=82) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
+
+
+def _decode(lib, q=16, kc=32, vc=48, sinks=64, ln=80, window=0, out=96, batch=2, max_len=100,
+            ws=128, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = lib.gptoss_attn_decode_workspace_bytes(batch, max_len, window)
+    return lib.gptoss_attn_decode(q, kc, vc, sinks, ln, window, out, batch, max_len, ws, ws_bytes,
+                                  None)
+
+
+def test_decode_argument_errors(lib):
+    c = _header_codes()
+    assert _decode(lib, kc=None) == c["GPTOSS_ATTN_ERR_NULL_PTR"]
+    assert _decode(lib, ws=None) == c["GPTOSS_ATTN_ERR_NULL_PTR"]
+    assert _decode(lib, batch=0, ws_bytes=1 << 20) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert _decode(lib, max_len=0, ws_bytes=1 << 20) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert _decode(lib, out=100) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
+    assert _decode(lib, ws=136) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
+    need = lib.gptoss_attn_decode_workspace_bytes(2, 100, 0)
+    assert need > 0
+    assert _decode(lib, ws_bytes=need - 1) == c["GPTOSS_ATTN_ERR_SMALL_WORKSPACE"]
+
+
+def test_workspace_query(lib):
+    assert lib.gptoss_attn_decode_workspace_bytes(0, 10, 0) == 0
+    assert lib.gptoss_attn_decode_workspace_bytes(1, 0, 0) == 0
+    full = lib.gptoss_attn_decode_workspace_bytes(64, 8192, 0)
+    slid = lib.gptoss_attn_decode_workspace_bytes(64, 8192, 128)
+    assert full >= slid > 0
+    # per (batch, head, split): 64 fp32 partial outputs + (max, sum)
+    assert full % (64 * 64 * (64 * 4 + 8)) == 0
+
+
+def test_python_binding_refuses_without_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    q = torch.zeros(1, 4, 64, 64, dtype=torch.bfloat16)
+    kv = torch.zeros(1, 4, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError):
+        gqa.prefill(q, kv, kv, torch.zeros(64), torch.zeros(1, 4, dtype=torch.int32), 0)

@@ -1,0 +1,177 @@
+"""GPU parity of the prefill kernel against the fp64 oracle, through the C ABI.
+
+Inputs come from the seeded generator (bf16 N(0,1) q/k/v, fp32 N(0,1)
+sinks); both sides see the same bf16 values. Bars: max-abs 2e-2 and
+mean-abs 2e-3 on the bf16 output.
+"""
+import numpy as np
+import pytest
+import torch
+
+import attention_gqa_b200 as gqa
+import oracle
+import synth
+from tests._util import bits_to_dev, compare, dev_to_f64
+
+pytestmark = pytest.mark.gpu
+
+NQ, NKV, D = 64, 8, 64
+
+
+def _inputs(config, layer, B, S, pos_offset=0):
+    x = synth.make_prefill_inputs(config, layer, B, S)
+    x["pos"] = (x["pos"] + pos_offset).astype(np.int32)
+    return x
+
+
+def _run_gpu(x, window, check=True):
+    out = gqa.prefill(bits_to_dev(x["q"]), bits_to_dev(x["k"]), bits_to_dev(x["v"]),
+                      torch.from_numpy(x["sinks"]).cuda(), torch.from_numpy(x["pos"]).cuda(),
+                      window)
+    if check:
+        gqa.check()
+    return out
+
+
+def _oracle_full(x, window):
+    return oracle.prefill(synth.bf16_bits_to_f64(x["q"]), synth.bf16_bits_to_f64(x["k"]),
+                          synth.bf16_bits_to_f64(x["v"]), x["sinks"], x["pos"], window)
+
+
+def test_rope_table_matches_fp64_rotation(cuda_device):
+    """Table rows equal cos/sin of p * theta^(-2k/64) from the oracle's rotation."""
+    tab = gqa.rope_table().cpu().numpy().astype(np.float64)        # [P, 32, 2]
+    rng = np.random.default_rng(3)
+    ps = np.concatenate([[0, 1, 2, 4095, 4096, 65535, 131071], rng.integers(0, 131072, 57)])
+    eye = np.zeros((32, D))
+    eye[np.arange(32), np.arange(32)] = 1.0
+    for p in ps:
+        y = oracle.rope(eye, float(p))                               # row k: e_k rotated
+        cos_ref = y[np.arange(32), np.arange(32)]
+        sin_ref = y[np.arange(32), np.arange(32) + 32]
+        assert np.max(np.abs(tab[p, :, 0] - cos_ref)) < 1.2e-7, p
+        assert np.max(np.abs(tab[p, :, 1] - sin_ref)) < 1.2e-7, p
+
+
+@pytest.mark.parametrize("window", [0, 128])
+def test_tiny_config_full_compare(cuda_device, window):
+    """B=1, S=256, 64/8 heads, full causal and 128-token window."""
+    x = _inputs(1, 0 if window == 0 else 1, 1, 256)
+    got = dev_to_f64(_run_gpu(x, window))
+    compare(got, _oracle_full(x, window), "S=256 W=%d" % window)
+
+
+@pytest.mark.parametrize("B,S", [(1, 1), (2, 2), (1, 15), (3, 16), (1, 17), (2, 33), (1, 127),
+                                 (1, 128), (2, 129), (1, 200), (1, 383)])
+@pytest.mark.parametrize("window", [0, 1, 5, 128, 300])
+def test_ragged_shapes_and_windows(cuda_device, B, S, window):
+    """Tails that are not multiples of the 32-token or 128-key tiles, odd batches,
+    windows shorter than, equal to and longer than the tiles."""
+    x = _inputs(100 + S, window, B, S)
+    got = dev_to_f64(_run_gpu(x, window))
+    compare(got, _oracle_full(x, window), "B=%d S=%d W=%d" % (B, S, window))
+
+
+def test_large_positions(cuda_device):
+    """Positions near the top of the table: the angles reach 1.3e5 rad."""
+    x = _inputs(7, 0, 1, 300, pos_offset=131072 - 300)
+    got = dev_to_f64(_run_gpu(x, 0))
+    compare(got, _oracle_full(x, 0), "large positions")
+
+
+def test_arbitrary_positions(cuda_device):
+    """Positions are only rotation angles: a random permutation of large values."""
+    x = _inputs(8, 0, 2, 160)
+    rng = np.random.default_rng(11)
+    x["pos"] = rng.integers(0, 131072, size=x["pos"].shape).astype(np.int32)
+    got = dev_to_f64(_run_gpu(x, 0))
+    compare(got, _oracle_full(x, 0), "random positions")
+
+
+@pytest.mark.parametrize("sink_value", [-np.inf, -30.0, 0.0, 12.0])
+def test_sink_extremes(cuda_device, sink_value):
+    """sigma = -inf (plain softmax), very negative, zero and dominant sinks."""
+    x = _inputs(9, 0, 1, 200)
+    x["sinks"] = np.full(NQ, sink_value, dtype=np.float32)
+    for window in (0, 3):
+        got = dev_to_f64(_run_gpu(x, window))
+        compare(got, _oracle_full(x, window), "sink=%s W=%d" % (sink_value, window))
+
+
+def test_scaled_inputs_trigger_rescale(cuda_device):
+    """Large scores make the running max climb many times across key tiles."""
+    x = _inputs(10, 0, 1, 700)
+    q = synth.bf16_bits_to_f64(x["q"]) * 4.0
+    x["q"] = synth.f32_to_bf16_bits(q.astype(np.float32))
+    got = dev_to_f64(_run_gpu(x, 0))
+    compare(got, _oracle_full(x, 0), "scaled q")
+
+
+def test_output_canaries(cuda_device):
+    """Nothing is written outside the output tensor."""
+    x = _inputs(12, 0, 2, 77)
+    n = 2 * 77 * NQ * D
+    buf = torch.full((n + 4096,), 1.5, dtype=torch.bfloat16, device="cuda")
+    out = buf[2048:2048 + n].view(2, 77, NQ, D)
+    gqa.prefill(bits_to_dev(x["q"]), bits_to_dev(x["k"]), bits_to_dev(x["v"]),
+                torch.from_numpy(x["sinks"]).cuda(), torch.from_numpy(x["pos"]).cuda(), 0, out=out)
+    gqa.check()
+    assert torch.all(buf[:2048] == 1.5) and torch.all(buf[2048 + n:] == 1.5)
+    compare(dev_to_f64(out), _oracle_full(x, 0), "canary run")
+
+
+def test_bad_position_is_reported(cuda_device):
+    x = _inputs(13, 0, 1, 40)
+    x["pos"][0, 5] = 131072
+    _run_gpu(x, 0, check=False)
+    with pytest.raises(gqa.GptossAttnError) as e:
+        gqa.check()
+    assert e.value.status == -10
+    gqa.check()  # cleared
+
+
+def test_host_buffers_end_to_end(cuda_device):
+    """CPU tensors in, CPU tensor out (the copies are part of the call)."""
+    x = _inputs(14, 0, 1, 96)
+    def host(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    out = gqa.prefill(host(x["q"]), host(x["k"]), host(x["v"]), torch.from_numpy(x["sinks"]),
+                      torch.from_numpy(x["pos"]), 0)
+    assert out.device.type == "cpu"
+    got = synth.bf16_bits_to_f64(out.view(torch.int16).numpy().view(np.uint16))
+    compare(got, _oracle_full(x, 0), "host buffers")
+
+
+@pytest.mark.parametrize("layer,window", [(0, 128), (1, 0)])
+def test_prefill_4096_two_layers(cuda_device, layer, window):
+    """B=1, S=4096: a 128-window layer then a full-causal layer, reseeded per layer."""
+    x = _inputs(2, layer, 1, 4096)
+    got = dev_to_f64(_run_gpu(x, window))
+    compare(got, _oracle_full(x, window), "S=4096 W=%d" % window)
+
+
+def _sample_rows(B, S, seed, n_random=128):
+    rng = np.random.default_rng(seed)
+    toks = set(range(min(256, S))) | set(range(max(0, S - 256), S)) | set(range(120, min(137, S)))
+    toks |= set(rng.integers(0, S, n_random).tolist())
+    return [(b, t) for b in range(B) for t in sorted(toks)]
+
+
+@pytest.mark.parametrize("config,B,S,layer,window", [
+    (3, 4, 16384, 0, 128), (3, 4, 16384, 1, 0),
+    (5, 1, 131072, 0, 0), (5, 1, 131072, 1, 128)])
+def test_full_size_sampled_rows(cuda_device, config, B, S, layer, window):
+    """Full-size layers in the launch configuration the bench times; the oracle
+    checks the first and last 256 tokens, the window edge and random tokens of
+    every sequence, all 64 heads."""
+    x = _inputs(config, layer, B, S)
+    out = _run_gpu(x, window)
+    rows = _sample_rows(B, S, config * 100 + layer)
+    idx_b = torch.tensor([r[0] for r in rows], device="cuda")
+    idx_t = torch.tensor([r[1] for r in rows], device="cuda")
+    got = dev_to_f64(out[idx_b, idx_t])
+    del out
+    q_rows = synth.bf16_bits_to_f64(np.stack([x["q"][b, t] for b, t in rows]))
+    ref = oracle.prefill_rows(q_rows, synth.bf16_bits_to_f64(x["k"]),
+                              synth.bf16_bits_to_f64(x["v"]), x["sinks"], x["pos"], window, rows)
+    compare(got, ref, "config %d layer %d" % (config, layer))

@@ -275,7 +275,8 @@ def test_rows_subset_matches_full():
     q, k, v, sinks, pos = _rand_inputs(800, 2, 50)
     full = oracle.prefill(q, k, v, sinks, pos, 7)
     rows = [(1, 49), (0, 0), (1, 3), (0, 20)]
-    sub = oracle.prefill_rows(q, k, v, sinks, pos, 7, rows)
+    q_rows = np.stack([q[b, i] for b, i in rows])
+    sub = oracle.prefill_rows(q_rows, k, v, sinks, pos, 7, rows)
     for n, (b, i) in enumerate(rows):
         assert np.array_equal(sub[n], full[b, i])
 
