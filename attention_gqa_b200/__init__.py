@@ -20,7 +20,7 @@ import os
 
 import torch
 
-__all__ = ["prefill", "decode", "decode_workspace_bytes", "check", "init", "rope_table",
+__all__ = ["prefill", "decode", "prefill_workspace_bytes", "decode_workspace_bytes", "check", "init", "rope_table",
            "library_path", "GptossAttnError", "NUM_HEADS", "NUM_KV_HEADS", "HEAD_DIM",
            "MAX_POSITION"]
 
@@ -62,7 +62,9 @@ def _load():
     lib.gptoss_attn_init.restype = i32
     lib.gptoss_attn_rope_table.argtypes = [ctypes.POINTER(vp)]
     lib.gptoss_attn_rope_table.restype = i32
-    lib.gptoss_attn_prefill.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, vp]
+    lib.gptoss_attn_prefill_workspace_bytes.argtypes = [i32, i32]
+    lib.gptoss_attn_prefill_workspace_bytes.restype = sz
+    lib.gptoss_attn_prefill.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, vp, sz, vp]
     lib.gptoss_attn_prefill.restype = i32
     lib.gptoss_attn_decode_workspace_bytes.argtypes = [i32, i32, i32]
     lib.gptoss_attn_decode_workspace_bytes.restype = sz
@@ -135,7 +137,12 @@ def rope_table() -> torch.Tensor:
     return view.clone()
 
 
-def prefill(q, k, v, sinks, pos, window: int = 0, out=None, stream=None) -> torch.Tensor:
+def prefill_workspace_bytes(batch: int, seqlen: int) -> int:
+    return int(_load().gptoss_attn_prefill_workspace_bytes(batch, seqlen))
+
+
+def prefill(q, k, v, sinks, pos, window: int = 0, out=None, workspace=None,
+            stream=None) -> torch.Tensor:
     """Causal grouped-query attention with sinks over whole sequences.
 
     Host (CPU) tensors are copied to the current CUDA device first and the
@@ -151,7 +158,7 @@ def prefill(q, k, v, sinks, pos, window: int = 0, out=None, stream=None) -> torc
                 res = prefill(q.to(device, non_blocking=True), k.to(device, non_blocking=True),
                               v.to(device, non_blocking=True),
                               sinks.to(device, non_blocking=True),
-                              pos.to(device, non_blocking=True), window, None, s)
+                              pos.to(device, non_blocking=True), window, None, workspace, s)
                 if out is None:
                     out = torch.empty(res.shape, dtype=res.dtype, pin_memory=True)
                 out.copy_(res, non_blocking=True)
@@ -174,8 +181,12 @@ def prefill(q, k, v, sinks, pos, window: int = 0, out=None, stream=None) -> torc
         raise ValueError("pos must be [B, S]")
     dev_out = out if (out is not None and out.device.type == "cuda") else torch.empty(
         (B, S, NUM_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=device)
+    if workspace is None:
+        workspace = torch.empty(prefill_workspace_bytes(B, S), dtype=torch.uint8, device=device)
     st = lib.gptoss_attn_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), sinks.data_ptr(),
                                  pos.data_ptr(), int(window), dev_out.data_ptr(), B, S,
+                                 workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(),
                                  _stream_handle(stream))
     _raise(st, "gptoss_attn_prefill")
     return dev_out

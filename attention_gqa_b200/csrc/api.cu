@@ -3,7 +3,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/gptoss_attn.h"
+#include "gptoss_attn.h"
 #include "internal.h"
 #include "tmap.h"
 
@@ -16,6 +16,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceState {
   int* err = nullptr;       // 4-byte error word
   float2* rope = nullptr;   // [kMaxPosition][32]
+  int num_sms = 0;
 };
 
 std::mutex g_mutex;
@@ -36,6 +37,9 @@ int current_device(int* dev) {
 int ensure_state(int dev, bool need_rope) {
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceState& st = g_state[dev];
+  if (st.num_sms == 0 &&
+      cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return GPTOSS_ATTN_ERR_NO_DEVICE;
   if (!st.err) {
     int* e = nullptr;
     if (cudaMalloc(&e, sizeof(int)) != cudaSuccess) return GPTOSS_ATTN_ERR_ALLOC;
@@ -101,15 +105,23 @@ int gptoss_attn_rope_table(const void** table) {
   return GPTOSS_ATTN_OK;
 }
 
+size_t gptoss_attn_prefill_workspace_bytes(int batch, int seqlen) {
+  if (batch < 1 || seqlen < 1 || seqlen > kMaxPosition || batch > 65535) return 0;
+  return static_cast<size_t>(batch) * seqlen * kNumKvHeads * kHeadDim * 2;
+}
+
 int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float* sinks,
                         const int32_t* pos, int window, void* out, int batch, int seqlen,
-                        cudaStream_t stream) {
-  if (!q || !k || !v || !sinks || !pos || !out) return GPTOSS_ATTN_ERR_NULL_PTR;
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !k || !v || !sinks || !pos || !out || !workspace) return GPTOSS_ATTN_ERR_NULL_PTR;
   if (batch < 1 || seqlen < 1 || seqlen > kMaxPosition || batch > 65535)
     return GPTOSS_ATTN_ERR_BAD_SHAPE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-      (reinterpret_cast<uintptr_t>(sinks) & 3u) || (reinterpret_cast<uintptr_t>(pos) & 3u))
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(sinks) & 3u) ||
+      (reinterpret_cast<uintptr_t>(pos) & 3u))
     return GPTOSS_ATTN_ERR_BAD_ALIGN;
+  if (workspace_bytes < gptoss_attn_prefill_workspace_bytes(batch, seqlen))
+    return GPTOSS_ATTN_ERR_SMALL_WORKSPACE;
   int dev = 0;
   int st = current_device(&dev);
   if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, true);
@@ -124,10 +136,14 @@ int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float
   const uint64_t kstr[3] = {kHeadDim * 2, kNumKvHeads * kHeadDim * 2,
                             S * kNumKvHeads * kHeadDim * 2};
   const uint32_t kbox[4] = {kHeadDim, 1, 128, 1};
+  const uint32_t kbox_band[4] = {kHeadDim, 1, 144, 1};
+  // the attention kernels read the rotated keys from the workspace
   if (!make_tmap_bf16_4d(&maps.q, q, qdims, qstr, qbox) ||
       !make_tmap_bf16_4d(&maps.o, out, qdims, qstr, qbox) ||
-      !make_tmap_bf16_4d(&maps.k, k, kdims, kstr, kbox) ||
-      !make_tmap_bf16_4d(&maps.v, v, kdims, kstr, kbox))
+      !make_tmap_bf16_4d(&maps.k, workspace, kdims, kstr, kbox) ||
+      !make_tmap_bf16_4d(&maps.v, v, kdims, kstr, kbox) ||
+      !make_tmap_bf16_4d(&maps.k_band, workspace, kdims, kstr, kbox_band) ||
+      !make_tmap_bf16_4d(&maps.v_band, v, kdims, kstr, kbox_band))
     return GPTOSS_ATTN_ERR_TENSOR_MAP;
 
   PrefillArgs args;
@@ -137,8 +153,14 @@ int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float
   args.err = g_state[dev].err;
   args.batch = batch;
   args.seqlen = seqlen;
-  args.window = window > 0 ? window : 0;
+  // A window covering the whole sequence is full causal.
+  args.window = (window > 0 && window < seqlen) ? window : 0;
   args.n_qtiles = (seqlen + 31) / 32;
+  args.n_items = prefill_items(batch, seqlen, args.window);
+  args.grid = g_state[dev].num_sms;
+  if (launch_rope_keys(k, pos, args.rope, workspace, static_cast<int64_t>(batch) * seqlen,
+                       args.grid * 8, args.err, stream) != cudaSuccess)
+    return GPTOSS_ATTN_ERR_LAUNCH;
   return launch_prefill(maps, args, stream) == cudaSuccess ? GPTOSS_ATTN_OK
                                                            : GPTOSS_ATTN_ERR_LAUNCH;
 }

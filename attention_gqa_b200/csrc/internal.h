@@ -33,17 +33,29 @@ struct PrefillArgs {
   int seqlen;
   int window;           // <= 0: full causal
   int n_qtiles;         // ceil(seqlen / 32)
+  int n_items;          // work items (prefill_items)
+  int grid;             // persistent CTAs (the device's SM count)
 };
 
 struct PrefillMaps {
-  CUtensorMap q, k, v, o;
+  CUtensorMap q, k, v, o;   // q/o boxes (64, 8, 16, 1); k/v boxes (64, 1, 128, 1)
+  CUtensorMap k_band, v_band;  // k/v boxes (64, 1, 144, 1) for the narrow-band kernel
 };
+
+// True when the narrow-band kernel (0 < window <= 128) serves the layer.
+bool prefill_uses_band(int window);
+// Work items of one prefill launch.
+int prefill_items(int batch, int seqlen, int window);
 
 // Launches the prefill kernel; returns a cudaError_t.
 cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream);
 
 // Fills the rotary table [kMaxPosition][32] of (cos, sin).
 cudaError_t launch_rope_table(float2* table, cudaStream_t stream);
+
+// Rotates the key rows of k [n_tokens][8][64] (bf16) by pos[token] into k_rot.
+cudaError_t launch_rope_keys(const void* k, const int32_t* pos, const float2* table, void* k_rot,
+                             int64_t n_tokens, int grid_cap, int* err, cudaStream_t stream);
 
 struct DecodeArgs {
   const uint16_t* q;       // [B][64][64] bf16, un-rotated

@@ -5,22 +5,29 @@
 // "Grouped-query attention", "Partial RoPE", "Learnable attention sink",
 // "Sliding-window attention"; llm-atlas field tables for the constants).
 //
-// One CTA handles one work item: batch b, key/value head g, and 32 query
-// tokens. The 8 query heads of group g are packed into the M dimension, so a
-// work item is two M=128 tiles (16 tokens x 8 heads each) that share every
-// K/V tile loaded. Roles (512 threads):
-//   warp 0       TMA producer: Q once, then K/V tiles of 128 keys through a
-//                kStages-deep ring.
-//   warp 1       TMEM owner and tcgen05 issuer (one thread): S = Q K^T
-//                (SS, K-major) and O += P V (A = P from TMEM, B = V MN-major).
-//   warps 4-7    softmax for M tile 0 (thread = TMEM lane = one query row)
-//   warps 8-11   softmax for M tile 1
-//   warps 12-15  RoPE: rotate Q rows and every K tile in shared memory.
-// Online softmax in log2 units with the running max seeded by the sink,
-// m0 = sigma*log2(e) and l0 = 1; O is rescaled only when the max grows by
-// more than 2^8 (the result is exact because O and l share the reference).
-// Tiles wholly outside the causal/window band are never visited; only
-// boundary tiles evaluate the mask per element.
+// Work item: batch b, key/value head g, 32 query tokens. The 8 query heads of
+// group g are packed into the M dimension, so an item is two M=128 tiles
+// (16 tokens x 8 heads) sharing every K/V tile. CTAs are persistent (one per
+// SM) and walk a static "snake" order over the items sorted longest first,
+// which balances the causal triangle without a global counter.
+//
+// Roles (512 threads, four warpgroups):
+//   WG0 warp 0    TMA producer: Q per item into a 2-slot buffer, K/V tiles of
+//                 128 keys through a kStages-deep ring.
+//   WG0 warp 1    TMEM owner and tcgen05 issuer (one thread): S = Q K^T
+//                 (SS, K-major) and O += P V (A = P from TMEM, B = V MN-major).
+//   WG0 warps 2-3 RoPE: rotate the Q rows of each item in shared memory, from
+//                 an fp64-built (cos, sin) table. Keys arrive already rotated
+//                 (a pre-pass rotates each key once per layer).
+//   WG1, WG2      softmax for M tile 0 / 1 (thread = TMEM lane = one query row):
+//                 one 128-column TMEM load per tile, sink-seeded online softmax
+//                 in log2 units, bf16 P written back over S.
+//   WG3           epilogue: O / l -> bf16 -> swizzled staging -> TMA store.
+// TMEM (512 columns): S0 [0,128), S1 [128,256) with P aliased on their first
+// 64 columns; O[m][item parity] at 256 + 64*(2*parity + m), so the next
+// item's P.V never waits for the previous item's epilogue.
+// The running max starts at sigma*log2(e) with l = 1; O is rescaled only when
+// the max grows by more than 2^8 (exact: O and l share the reference).
 #include <cmath>
 
 #include "internal.h"
@@ -37,33 +44,42 @@ constexpr int kThreads = 512;
 constexpr uint32_t kTileBytes = 128 * 128;  // 128 rows of 64 bf16
 
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns of M tile m: S (fp32, 128 columns) with P (bf16) aliased on
-// its first 64, and the O accumulator (fp32, 64 columns).
 __host__ __device__ constexpr uint32_t tmem_s(int m) { return m ? 128u : 0u; }
-__host__ __device__ constexpr uint32_t tmem_o(int m) { return m ? 320u : 256u; }
+__host__ __device__ constexpr uint32_t tmem_o(int m, int ob) {
+  return 256u + 64u * static_cast<uint32_t>(2 * ob + m);
+}
+
+// Register budgets after the warpgroup split; launch is 512 x 128.
+constexpr uint32_t kRegsLight = 88;     // WG0 and WG3
+constexpr uint32_t kRegsSoftmax = 168;  // WG1 and WG2
+static_assert(2 * 128 * kRegsLight + 2 * 128 * kRegsSoftmax <= 512 * 128, "register split");
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kScaleLog2 = 0.125f * kLog2e;  // 1/sqrt(64) * log2(e)
 constexpr float kRescaleThreshold = 8.0f;      // log2 units
 
 enum : int {
-  BAR_Q_FULL = 0,
-  BAR_Q_READY,
-  BAR_K_FULL,
-  BAR_V_FULL = BAR_K_FULL + kStages,
-  BAR_K_READY = BAR_V_FULL + kStages,
-  BAR_KV_EMPTY = BAR_K_READY + kStages,
-  BAR_S_FULL = BAR_KV_EMPTY + kStages,
-  BAR_P_FULL = BAR_S_FULL + 2,
-  BAR_O_FULL = BAR_P_FULL + 2,
-  BAR_MMA_DONE = BAR_O_FULL + 2,
+  BAR_Q_FULL = 0,                        // [2] slot loaded
+  BAR_Q_READY = BAR_Q_FULL + 2,          // [2] slot rotated
+  BAR_Q_EMPTY = BAR_Q_READY + 2,         // [2] slot's output stored
+  BAR_K_FULL = BAR_Q_EMPTY + 2,          // [kStages]
+  BAR_V_FULL = BAR_K_FULL + kStages,     // [kStages]
+  BAR_KV_EMPTY = BAR_V_FULL + kStages,   // [kStages]
+  BAR_S_FULL = BAR_KV_EMPTY + kStages,   // [2] per M tile
+  BAR_P_FULL = BAR_S_FULL + 2,           // [2]
+  BAR_O_FULL = BAR_P_FULL + 2,           // [4] m*2 + parity
+  BAR_O_EMPTY = BAR_O_FULL + 4,          // [4]
+  BAR_L_FULL = BAR_O_EMPTY + 4,          // [2]
+  BAR_L_EMPTY = BAR_L_FULL + 2,          // [2]
+  BAR_MMA_DONE = BAR_L_EMPTY + 2,
   NUM_BARS
 };
 
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;
+constexpr uint32_t kOffQ = 0;  // [2 slots][2 halves] tiles
+constexpr uint32_t kOffK = kOffQ + 4 * kTileBytes;
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
-constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+constexpr uint32_t kOffL = kOffV + kStages * kTileBytes;  // float [2][128]
+constexpr uint32_t kOffBar = kOffL + 2 * 128 * 4;
 constexpr uint32_t kOffMisc = kOffBar + NUM_BARS * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
 
@@ -75,7 +91,36 @@ struct Ctx {
   __device__ bool wait(int i, uint32_t parity) const {
     return mbar_wait(bar(i), parity, abort_flag, err, kErrTimeout, kWaitTimeoutNs);
   }
+  __device__ bool wait_warp(int i, uint32_t parity) const {
+    return mbar_wait_warp(bar(i), parity, abort_flag, err, kErrTimeout, kWaitTimeoutNs);
+  }
+  __device__ uint32_t q_tile(int slot, int m) const {
+    return sbase + kOffQ + static_cast<uint32_t>(2 * slot + m) * kTileBytes;
+  }
 };
+
+struct Item {
+  int b, g, q0, jt0, n_tiles;
+};
+
+// The k-th item of CTA `cta` in snake order over items sorted longest first
+// (query tile descending, then kv head, then batch); false past the end.
+__device__ __forceinline__ bool item_for(const PrefillArgs& a, int k, int cta, Item* it) {
+  const int grid = static_cast<int>(gridDim.x);
+  const int idx = (k & 1) ? (k + 1) * grid - 1 - cta : k * grid + cta;
+  if (idx >= a.n_items) return false;
+  const int per_tile = kNumKvHeads * a.batch;
+  const int qt = a.n_qtiles - 1 - idx / per_tile;
+  const int rem = idx % per_tile;
+  it->g = rem % kNumKvHeads;
+  it->b = rem / kNumKvHeads;
+  it->q0 = qt * kBlockQ;
+  const int qlast = min(it->q0 + kBlockQ - 1, a.seqlen - 1);
+  const int klo = a.window > 0 ? max(0, it->q0 - a.window + 1) : 0;
+  it->jt0 = klo / kBlockN;
+  it->n_tiles = qlast / kBlockN - it->jt0 + 1;
+  return true;
+}
 
 __device__ __forceinline__ int load_position(const PrefillArgs& a, int b, int t) {
   int p = __ldg(a.pos + static_cast<size_t>(b) * a.seqlen + t);
@@ -87,15 +132,15 @@ __device__ __forceinline__ int load_position(const PrefillArgs& a, int b, int t)
 }
 
 // Rotate one 64-element row stored at `row` (128 bytes, 128B-swizzled with
-// row index r) by the table entry of position p, in place.
+// row index r) by the table entry `cs` of its position, in place.
 __device__ __forceinline__ void rope_row(uint8_t* row, int r, const float2* __restrict__ cs) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     uint4* plo = reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4));
     uint4* phi = reinterpret_cast<uint4*>(row + (((c + 4) ^ (r & 7)) << 4));
-    const uint4 a = *plo, h = *phi;
     const float4* t4 = reinterpret_cast<const float4*>(cs + 8 * c);
     const float4 t0 = __ldg(t4 + 0), t1 = __ldg(t4 + 1), t2 = __ldg(t4 + 2), t3 = __ldg(t4 + 3);
+    const uint4 a = *plo, h = *phi;
     const float cv[8] = {t0.x, t0.z, t1.x, t1.z, t2.x, t2.z, t3.x, t3.z};
     const float sv[8] = {t0.y, t0.w, t1.y, t1.w, t2.y, t2.w, t3.y, t3.w};
     const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
@@ -114,6 +159,10 @@ __device__ __forceinline__ void rope_row(uint8_t* row, int r, const float2* __re
   }
 }
 
+__device__ __forceinline__ bool key_visible(int kj, int tq, int W) {
+  return kj <= tq && (W <= 0 || kj > tq - W);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs args) {
   extern __shared__ uint8_t smem_raw[];
@@ -124,33 +173,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   ctx.abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   ctx.err = args.err;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  float* l_smem = reinterpret_cast<float*>(smem + kOffL);
 
   const int warp = static_cast<int>(threadIdx.x >> 5);
   const int lane = static_cast<int>(threadIdx.x & 31);
-  const int qt = args.n_qtiles - 1 - static_cast<int>(blockIdx.x);  // longest rows first
-  const int g = static_cast<int>(blockIdx.y);
-  const int b = static_cast<int>(blockIdx.z);
+  const int cta = static_cast<int>(blockIdx.x);
   const int S = args.seqlen;
   const int W = args.window;
-  const int q0 = qt * kBlockQ;
-  const int qlast = min(q0 + kBlockQ - 1, S - 1);
-  const int klo = W > 0 ? max(0, q0 - W + 1) : 0;
-  const int jt0 = klo / kBlockN;
-  const int n_tiles = qlast / kBlockN - jt0 + 1;
 
   if (threadIdx.x == 0) {
-    mbar_init(ctx.bar(BAR_Q_FULL), 1);
-    mbar_init(ctx.bar(BAR_Q_READY), 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(ctx.bar(BAR_Q_FULL + i), 1);
+      mbar_init(ctx.bar(BAR_Q_READY + i), 2);
+      mbar_init(ctx.bar(BAR_Q_EMPTY + i), 1);
+      mbar_init(ctx.bar(BAR_S_FULL + i), 1);
+      mbar_init(ctx.bar(BAR_P_FULL + i), 4);
+      mbar_init(ctx.bar(BAR_L_FULL + i), 4);
+      mbar_init(ctx.bar(BAR_L_EMPTY + i), 4);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(ctx.bar(BAR_K_FULL + s), 1);
       mbar_init(ctx.bar(BAR_V_FULL + s), 1);
-      mbar_init(ctx.bar(BAR_K_READY + s), 4);
       mbar_init(ctx.bar(BAR_KV_EMPTY + s), 1);
     }
-    for (int m = 0; m < 2; ++m) {
-      mbar_init(ctx.bar(BAR_S_FULL + m), 1);
-      mbar_init(ctx.bar(BAR_P_FULL + m), 4);
-      mbar_init(ctx.bar(BAR_O_FULL + m), 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(ctx.bar(BAR_O_FULL + i), 1);
+      mbar_init(ctx.bar(BAR_O_EMPTY + i), 4);
     }
     mbar_init(ctx.bar(BAR_MMA_DONE), 1);
     // A pipeline timeout earlier left the error word set: skip the work.
@@ -166,259 +214,666 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const bool skip = *ctx.abort_flag != 0;
+  const int wg = warp >> 2;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0 && !skip) {
-      prefetch_tensormap(&maps.q);
-      prefetch_tensormap(&maps.k);
-      prefetch_tensormap(&maps.v);
-      prefetch_tensormap(&maps.o);
-      mbar_arrive_expect_tx(ctx.bar(BAR_Q_FULL), 2 * kTileBytes);
-      tma_load_4d(ctx.sbase + kOffQ, &maps.q, ctx.bar(BAR_Q_FULL), 0, g * kGroup, q0, b);
-      tma_load_4d(ctx.sbase + kOffQ + kTileBytes, &maps.q, ctx.bar(BAR_Q_FULL), 0, g * kGroup,
-                  q0 + kTokensPerM, b);
-      int issued = 0;
-      for (int it = 0; it < n_tiles; ++it) {
-        const int s = it % kStages;
-        if (it >= kStages && !ctx.wait(BAR_KV_EMPTY + s, ((it / kStages) - 1) & 1)) break;
-        const int kb = (jt0 + it) * kBlockN;
-        mbar_arrive_expect_tx(ctx.bar(BAR_K_FULL + s), kTileBytes);
-        tma_load_4d(ctx.sbase + kOffK + s * kTileBytes, &maps.k, ctx.bar(BAR_K_FULL + s), 0, g, kb,
-                    b);
-        mbar_arrive_expect_tx(ctx.bar(BAR_V_FULL + s), kTileBytes);
-        tma_load_4d(ctx.sbase + kOffV + s * kTileBytes, &maps.v, ctx.bar(BAR_V_FULL + s), 0, g, kb,
-                    b);
-        issued = it + 1;
-      }
-      if (*ctx.abort_flag) {
-        // Let every copy this CTA started land before its shared memory is released.
-        volatile int never = 0;
-        mbar_wait(ctx.bar(BAR_Q_FULL), 0, &never, nullptr, 0, kWaitTimeoutNs);
-        for (int it = max(0, issued - kStages); it < issued; ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          mbar_wait(ctx.bar(BAR_K_FULL + s), ph, &never, nullptr, 0, kWaitTimeoutNs);
-          mbar_wait(ctx.bar(BAR_V_FULL + s), ph, &never, nullptr, 0, kWaitTimeoutNs);
+  if (wg == 0) {
+    setmaxnreg_dec<kRegsLight>();
+    if (warp == 0) {
+      // -------------------------------------------------------------- producer
+      if (lane == 0 && !skip) {
+        prefetch_tensormap(&maps.q);
+        prefetch_tensormap(&maps.k);
+        prefetch_tensormap(&maps.v);
+        int G = 0, n = 0, nq = 0;
+        Item it;
+        bool ok = true;
+        for (; ok && item_for(args, n, cta, &it); ++n) {
+          const int qs = n & 1;
+          if (n >= 2 && !(ok = ctx.wait(BAR_Q_EMPTY + qs, ((n >> 1) - 1) & 1))) break;
+          mbar_arrive_expect_tx(ctx.bar(BAR_Q_FULL + qs), 2 * kTileBytes);
+          tma_load_4d(ctx.q_tile(qs, 0), &maps.q, ctx.bar(BAR_Q_FULL + qs), 0, it.g * kGroup,
+                      it.q0, it.b);
+          tma_load_4d(ctx.q_tile(qs, 1), &maps.q, ctx.bar(BAR_Q_FULL + qs), 0, it.g * kGroup,
+                      it.q0 + kTokensPerM, it.b);
+          nq = n + 1;
+          for (int j = 0; j < it.n_tiles; ++j) {
+            const int s = G % kStages;
+            if (G >= kStages && !(ok = ctx.wait(BAR_KV_EMPTY + s, ((G / kStages) - 1) & 1)))
+              break;
+            const int kb = (it.jt0 + j) * kBlockN;
+            mbar_arrive_expect_tx(ctx.bar(BAR_K_FULL + s), kTileBytes);
+            tma_load_4d(ctx.sbase + kOffK + s * kTileBytes, &maps.k, ctx.bar(BAR_K_FULL + s), 0,
+                        it.g, kb, it.b);
+            mbar_arrive_expect_tx(ctx.bar(BAR_V_FULL + s), kTileBytes);
+            tma_load_4d(ctx.sbase + kOffV + s * kTileBytes, &maps.v, ctx.bar(BAR_V_FULL + s), 0,
+                        it.g, kb, it.b);
+            ++G;
+          }
         }
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && !skip) {
-      constexpr uint32_t idesc_qk = idesc_bf16(128, kBlockN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, kHeadDim, true);
-      auto issue_qk = [&](int m, int s) {
-        const uint32_t qa = ctx.sbase + kOffQ + m * kTileBytes;
-        const uint32_t ka = ctx.sbase + kOffK + s * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < kHeadDim / 16; ++kk)
-          mma_bf16_ss(tmem + tmem_s(m), sdesc_sw128(qa + 32 * kk), sdesc_sw128(ka + 32 * kk),
-                      idesc_qk, kk > 0 ? 1u : 0u);
-      };
-      auto issue_pv = [&](int m, int s, bool accumulate) {
-        const uint32_t va = ctx.sbase + kOffV + s * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk)
-          mma_bf16_ts(tmem + tmem_o(m), tmem + tmem_s(m) + 8 * kk, sdesc_sw128(va + 2048 * kk),
-                      idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
-      };
-      bool ok = ctx.wait(BAR_Q_READY, 0);
-      tc_fence_after_sync();
-      for (int it = 0; ok && it < n_tiles; ++it) {
-        const int s = it % kStages;
-        if (!(ok = ctx.wait(BAR_K_READY + s, (it / kStages) & 1))) break;
-        tc_fence_after_sync();
-        const int sp = (it + kStages - 1) % kStages;
-        if (it > 0) {
-          if (!(ok = ctx.wait(BAR_V_FULL + sp, ((it - 1) / kStages) & 1) &&
-                     ctx.wait(BAR_P_FULL + 0, (it - 1) & 1)))
-            break;
-          tc_fence_after_sync();
-          issue_pv(0, sp, it > 1);
-        }
-        issue_qk(0, s);
-        mma_commit(ctx.bar(BAR_S_FULL + 0));
-        if (it > 0) {
-          if (!(ok = ctx.wait(BAR_P_FULL + 1, (it - 1) & 1))) break;
-          tc_fence_after_sync();
-          issue_pv(1, sp, it > 1);
-          mma_commit(ctx.bar(BAR_KV_EMPTY + sp));
-        }
-        issue_qk(1, s);
-        mma_commit(ctx.bar(BAR_S_FULL + 1));
-      }
-      if (ok) {
-        const int last = n_tiles - 1;
-        const int sp = last % kStages;
-        if (ctx.wait(BAR_V_FULL + sp, (last / kStages) & 1) && ctx.wait(BAR_P_FULL + 0, last & 1)) {
-          tc_fence_after_sync();
-          issue_pv(0, sp, last > 0);
-          mma_commit(ctx.bar(BAR_O_FULL + 0));
-          if (ctx.wait(BAR_P_FULL + 1, last & 1)) {
-            tc_fence_after_sync();
-            issue_pv(1, sp, last > 0);
-            mma_commit(ctx.bar(BAR_KV_EMPTY + sp));
-            mma_commit(ctx.bar(BAR_O_FULL + 1));
+        if (*ctx.abort_flag) {
+          // Let every copy this CTA started land before its shared memory is released.
+          volatile int never = 0;
+          for (int i = max(0, nq - 2); i < nq; ++i)
+            mbar_wait(ctx.bar(BAR_Q_FULL + (i & 1)), (i >> 1) & 1, &never, nullptr, 0,
+                      kWaitTimeoutNs);
+          for (int i = max(0, G - kStages); i < G; ++i) {
+            mbar_wait(ctx.bar(BAR_K_FULL + i % kStages), (i / kStages) & 1, &never, nullptr, 0,
+                      kWaitTimeoutNs);
+            mbar_wait(ctx.bar(BAR_V_FULL + i % kStages), (i / kStages) & 1, &never, nullptr, 0,
+                      kWaitTimeoutNs);
           }
         }
       }
-      // Every MMA issued must finish before the tensor memory is released.
-      mma_commit(ctx.bar(BAR_MMA_DONE));
-      volatile int never = 0;
-      mbar_wait(ctx.bar(BAR_MMA_DONE), 0, &never, nullptr, 0, kWaitTimeoutNs);
+    } else if (warp == 1) {
+      // -------------------------------------------------------------- MMA issuer
+      if (lane == 0 && !skip) {
+        constexpr uint32_t idesc_qk = idesc_bf16(128, kBlockN, false);
+        constexpr uint32_t idesc_pv = idesc_bf16(128, kHeadDim, true);
+        auto issue_qk = [&](int m, int qs, int s) {
+          const uint32_t qa = ctx.q_tile(qs, m);
+          const uint32_t ka = ctx.sbase + kOffK + s * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kHeadDim / 16; ++kk)
+            mma_bf16_ss(tmem + tmem_s(m), sdesc_sw128(qa + 32 * kk), sdesc_sw128(ka + 32 * kk),
+                        idesc_qk, kk > 0 ? 1u : 0u);
+        };
+        auto issue_pv = [&](int m, int s, int ob, bool accumulate) {
+          const uint32_t va = ctx.sbase + kOffV + s * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBlockN / 16; ++kk)
+            mma_bf16_ts(tmem + tmem_o(m, ob), tmem + tmem_s(m) + 8 * kk,
+                        sdesc_sw128(va + 2048 * kk), idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+        };
+        // The P.V of the previous tile (global index pv_G, item pv_n) is issued
+        // interleaved with the current tile's Q.K^T on the other M tile.
+        int pv_G = -1, pv_n = 0;
+        bool pv_first = false, pv_last = false;
+        auto do_pv = [&](int m) -> bool {
+          const int s = pv_G % kStages;
+          if (m == 0 && !ctx.wait(BAR_V_FULL + s, (pv_G / kStages) & 1)) return false;
+          if (!ctx.wait(BAR_P_FULL + m, pv_G & 1)) return false;
+          if (pv_first && pv_n >= 2 &&
+              !ctx.wait(BAR_O_EMPTY + 2 * m + (pv_n & 1), ((pv_n >> 1) - 1) & 1))
+            return false;
+          tc_fence_after_sync();
+          issue_pv(m, s, pv_n & 1, !pv_first);
+          if (m == 1) mma_commit(ctx.bar(BAR_KV_EMPTY + s));
+          if (pv_last) mma_commit(ctx.bar(BAR_O_FULL + 2 * m + (pv_n & 1)));
+          return true;
+        };
+        int G = 0, n = 0;
+        Item it;
+        bool ok = true;
+        for (; ok && item_for(args, n, cta, &it); ++n) {
+          const int qs = n & 1;
+          if (!(ok = ctx.wait(BAR_Q_FULL + qs, (n >> 1) & 1) &&
+                     ctx.wait(BAR_Q_READY + qs, (n >> 1) & 1)))
+            break;
+          for (int j = 0; j < it.n_tiles; ++j, ++G) {
+            const int s = G % kStages;
+            if (!(ok = ctx.wait(BAR_K_FULL + s, (G / kStages) & 1))) break;
+            tc_fence_after_sync();
+            if (pv_G >= 0 && !(ok = do_pv(0))) break;
+            issue_qk(0, qs, s);
+            mma_commit(ctx.bar(BAR_S_FULL + 0));
+            if (pv_G >= 0 && !(ok = do_pv(1))) break;
+            issue_qk(1, qs, s);
+            mma_commit(ctx.bar(BAR_S_FULL + 1));
+            pv_G = G;
+            pv_n = n;
+            pv_first = j == 0;
+            pv_last = j == it.n_tiles - 1;
+          }
+        }
+        if (ok && pv_G >= 0 && do_pv(0)) do_pv(1);
+        // Every MMA issued must finish before the tensor memory is released.
+        mma_commit(ctx.bar(BAR_MMA_DONE));
+        volatile int never = 0;
+        mbar_wait(ctx.bar(BAR_MMA_DONE), 0, &never, nullptr, 0, kWaitTimeoutNs);
+      }
+    } else {
+      // -------------------------------------------------------------- RoPE
+      const int t = static_cast<int>(threadIdx.x) - 64;  // 0..63
+      int n = 0;
+      Item it;
+      bool ok = !skip;
+      for (; ok && item_for(args, n, cta, &it); ++n) {
+        const int qs = n & 1;
+        // positions first, so their latency overlaps the wait for the Q tile
+        int pq[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tok = it.q0 + (i >> 1) * kTokensPerM + ((t + 64 * (i & 1)) >> 3);
+          pq[i] = tok < S ? load_position(args, it.b, tok) : -1;
+        }
+        if (!(ok = ctx.wait_warp(BAR_Q_FULL + qs, (n >> 1) & 1))) break;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int row = t + 64 * (i & 1);
+          if (pq[i] >= 0)
+            rope_row(smem + kOffQ + (2 * qs + (i >> 1)) * kTileBytes + row * 128, row,
+                     args.rope + static_cast<size_t>(pq[i]) * kRopePairs);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ctx.bar(BAR_Q_READY + qs));
+      }
     }
-  } else if (warp >= 4 && warp < 12) {
+  } else if (wg == 1 || wg == 2) {
     // ---------------------------------------------------------------- softmax
-    const int m = (warp - 4) >> 2;  // M tile
-    const int wq = warp & 3;        // TMEM lane quarter of this warp
-    const int r = wq * 32 + lane;   // row of the M tile = TMEM lane
-    const int tq = q0 + m * kTokensPerM + (r >> 3);
-    const int h = g * kGroup + (r & 7);
-    const int tmin = q0 + m * kTokensPerM + wq * 4;  // tokens of this warp: tmin .. tmin+3
-    const int tmax = tmin + 3;
+    setmaxnreg_inc<kRegsSoftmax>();
+    const int m = wg - 1;          // M tile
+    const int wq = warp & 3;       // TMEM lane quarter of this warp
+    const int r = wq * 32 + lane;  // row of the M tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + tmem_s(m);
-    const uint32_t tO = tmem + lane_off + tmem_o(m);
-    const float sink = __ldg(args.sinks + h);
-    const bool sink_off = isinf(sink) && sink < 0.f;
-    float m_ref = sink_off ? -INFINITY : sink * kLog2e;
-    float l = sink_off ? 0.f : 1.f;
+    int G = 0, n = 0;
+    Item it;
     bool ok = !skip;
-    for (int it = 0; ok && it < n_tiles; ++it) {
-      if (!(ok = ctx.wait(BAR_S_FULL + m, it & 1))) break;
-      tc_fence_after_sync();
-      const int kb = (jt0 + it) * kBlockN;
-      const bool wmask = (kb + kBlockN - 1 > tmin) || (W > 0 && kb <= tmax - W);
-      // pass 1: row maximum of the visible scores
-      float mx = -INFINITY;
-#pragma unroll
-      for (int ch = 0; ch < kBlockN / 32; ++ch) {
-        uint32_t sv[32];
-        tmem_ld32(tS + ch * 32, sv);
+    for (; ok && item_for(args, n, cta, &it); ++n) {
+      const int tq = it.q0 + m * kTokensPerM + (r >> 3);
+      const int tmin = it.q0 + m * kTokensPerM + wq * 4;  // tokens of this warp: tmin .. tmin+3
+      const int tmax = tmin + 3;
+      const uint32_t tO = tmem + lane_off + tmem_o(m, n & 1);
+      const float sink = __ldg(args.sinks + it.g * kGroup + (r & 7));
+      const bool sink_off = isinf(sink) && sink < 0.f;
+      float m_ref = sink_off ? -INFINITY : sink * kLog2e;
+      float l = sink_off ? 0.f : 1.f;
+      for (int j = 0; j < it.n_tiles; ++j, ++G) {
+        if (!(ok = ctx.wait_warp(BAR_S_FULL + m, G & 1))) break;
+        tc_fence_after_sync();
+        const int kb = (it.jt0 + j) * kBlockN;
+        const bool wmask = (kb + kBlockN - 1 > tmin) || (W > 0 && kb <= tmax - W);
+        uint32_t sv[128];
+        tmem_ld128_split(tS, sv);
         if (wmask) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int kj = kb + ch * 32 + i;
-            const bool vis = kj <= tq && (W <= 0 || kj > tq - W);
-            mx = fmaxf(mx, vis ? __uint_as_float(sv[i]) : -INFINITY);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
+          for (int i = 0; i < 128; ++i)
+            if (!key_visible(kb + i, tq, W)) sv[i] = __float_as_uint(-INFINITY);
         }
-      }
-      mx *= kScaleLog2;
-      const float m_new = fmaxf(m_ref, mx);
-      float alpha = 1.f;
-      bool rescale = false;
-      if (it == 0) {
-        if (m_new > m_ref) {
-          l *= ex2_approx(m_ref - m_new);
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 128; i += 8) {
+          mx0 = fmax3(mx0, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+          mx1 = fmax3(mx1, __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]));
+          mx2 = fmax3(mx2, __uint_as_float(sv[i + 4]), __uint_as_float(sv[i + 5]));
+          mx3 = fmax3(mx3, __uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7]));
+        }
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * kScaleLog2;
+        const float m_new = fmaxf(m_ref, mx);
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          if (m_new > m_ref) {
+            l *= ex2_approx(m_ref - m_new);
+            m_ref = m_new;
+          }
+        } else if (m_new > m_ref + kRescaleThreshold) {
+          alpha = ex2_approx(m_ref - m_new);
+          l *= alpha;
           m_ref = m_new;
+          rescale = true;
         }
-      } else if (m_new > m_ref + kRescaleThreshold) {
-        alpha = ex2_approx(m_ref - m_new);
-        l *= alpha;
-        m_ref = m_new;
-        rescale = true;
-      }
-      if (__any_sync(0xffffffffu, rescale)) {
+        // probabilities, packed to bf16 in place: sv[i] <- (p[2i], p[2i+1]);
+        // scale-and-subtract and the row sum run on packed fp32 pairs
+        const float mr = m_ref == -INFINITY ? 0.f : m_ref;
+        const uint64_t c2 = f2_pack(kScaleLog2, kScaleLog2);
+        const uint64_t nm2 = f2_pack(-mr, -mr);
+        uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
-        for (int ch = 0; ch < kHeadDim / 32; ++ch) {
-          uint32_t ov[32];
-          tmem_ld32(tO + ch * 32, ov);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st32(tO + ch * 32, ov);
-        }
-      }
-      // pass 2: probabilities, row sum, bf16 P into the S columns
-      const float mr = m_ref == -INFINITY ? 0.f : m_ref;
-      float rs = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < kBlockN / 32; ++ch) {
-        uint32_t sv[32];
-        tmem_ld32(tS + ch * 32, sv);
-        uint32_t pw[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float x0 = fmaf(__uint_as_float(sv[2 * i]), kScaleLog2, -mr);
-          float x1 = fmaf(__uint_as_float(sv[2 * i + 1]), kScaleLog2, -mr);
-          if (wmask) {
-            const int kj = kb + ch * 32 + 2 * i;
-            if (!(kj <= tq && (W <= 0 || kj > tq - W))) x0 = -INFINITY;
-            if (!(kj + 1 <= tq && (W <= 0 || kj + 1 > tq - W))) x1 = -INFINITY;
-          }
+        for (int i = 0; i < 64; i += 2) {
+          float x0, x1, x2, x3;
+          f2_unpack(ffma2(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), c2,
+                          nm2),
+                    x0, x1);
+          f2_unpack(ffma2(f2_pack(__uint_as_float(sv[2 * i + 2]), __uint_as_float(sv[2 * i + 3])),
+                          c2, nm2),
+                    x2, x3);
           const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          rs += p0 + p1;
-          pw[i] = pack_bf16x2(p0, p1);
+          const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+          acc0 = fadd2(acc0, f2_pack(p0, p1));
+          acc1 = fadd2(acc1, f2_pack(p2, p3));
+          sv[i] = pack_bf16x2(p0, p1);
+          sv[i + 1] = pack_bf16x2(p2, p3);
         }
-        tmem_st16(tS + ch * 16, pw);
+        {
+          float a0, a1, a2, a3;
+          f2_unpack(acc0, a0, a1);
+          f2_unpack(acc1, a2, a3);
+          l += (a0 + a1) + (a2 + a3);
+        }
+        {
+          uint32_t pw[64];
+#pragma unroll
+          for (int i = 0; i < 64; ++i) pw[i] = sv[i];
+          tmem_st64(tS, pw);
+        }
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int ch = 0; ch < kHeadDim / 32; ++ch) {
+            uint32_t ov[32];
+            tmem_ld32(tO + ch * 32, ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32(tO + ch * 32, ov);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ctx.bar(BAR_P_FULL + m));
       }
-      l += rs;
+      if (!ok) break;
+      // hand the row sum to the epilogue
+      if (n >= 1 && !(ok = ctx.wait_warp(BAR_L_EMPTY + m, (n - 1) & 1))) break;
+      l_smem[m * 128 + r] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ctx.bar(BAR_L_FULL + m));
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    setmaxnreg_dec<kRegsLight>();
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    int n = 0;
+    Item it;
+    // Every thread runs every item (no early exit) so the named barrier
+    // below is always reached by all 128 threads; failed waits skip work.
+    for (; item_for(args, n, cta, &it); ++n) {
+      const int qs = n & 1;
+      const int ob = n & 1;
+      bool ok = !skip && !*ctx.abort_flag;
+#pragma unroll 1
+      for (int m = 0; m < 2; ++m) {
+        uint32_t ov[64];
+        const bool ok_o = ok && ctx.wait_warp(BAR_O_FULL + 2 * m + ob, (n >> 1) & 1);
+        if (ok_o) {
+          tc_fence_after_sync();
+          tmem_ld64(tmem + lane_off + tmem_o(m, ob), ov);
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(ctx.bar(BAR_O_EMPTY + 2 * m + ob));
+        }
+        const bool ok_l = ok_o && ctx.wait_warp(BAR_L_FULL + m, n & 1);
+        if (ok_l) {
+          const float l = l_smem[m * 128 + r];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(ctx.bar(BAR_L_EMPTY + m));
+          const float inv_l = 1.f / l;
+          uint8_t* stage = smem + kOffQ + (2 * qs + m) * kTileBytes;
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack_bf16x2(__uint_as_float(ov[8 * cc + 2 * e]) * inv_l,
+                                 __uint_as_float(ov[8 * cc + 2 * e + 1]) * inv_l);
+            *reinterpret_cast<uint4*>(stage + r * 128 + ((cc ^ (r & 7)) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+        ok = ok_l;
+      }
+      fence_async_smem();
+      named_barrier(1, 128);
+      if (threadIdx.x == 384) {
+        if (ok && !*ctx.abort_flag) {
+          for (int m = 0; m < 2; ++m)
+            if (it.q0 + m * kTokensPerM < S)
+              tma_store_4d(&maps.o, ctx.q_tile(qs, m), 0, it.g * kGroup, it.q0 + m * kTokensPerM,
+                           it.b);
+          tma_store_commit();
+          tma_store_wait_read();
+        }
+        mbar_arrive(ctx.bar(BAR_Q_EMPTY + qs));
+      }
+    }
+    if (threadIdx.x == 384) tma_store_wait_all();
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+
+// ============================================================================
+// Narrow-band kernel for sliding windows 0 < W <= 128 (the model's W = 128).
+//
+// Work item: batch b, kv head g, 16 query tokens = one M=128 tile. Query i
+// sees keys (i-W, i], so the whole item needs only the 144 keys
+// [q0-128, q0+16): one K/V span per item (TMA zero-fills rows before 0),
+// S = Q K^T with N = 144 and a single-tile softmax (no online rescaling).
+// Keys arrive already rotated; the RoPE warps rotate the item's Q rows.
+// Consecutive items alternate between the two softmax warpgroups so the
+// tensor core works on one item while the other's softmax runs. Each item's
+// Q, K and V share one ring stage; outputs go through a 4-slot staging ring
+// so the store of an item overlaps the next items' epilogues.
+namespace band {
+
+constexpr int kTokens = 16;
+constexpr int kSpan = 144;  // 128 keys before the tile + the tile's 16
+constexpr int kStages = 3;
+constexpr int kOutSlots = 4;  // output staging ring; a slot is reused 4 items later
+constexpr uint32_t kQBytes = 128 * 128;
+constexpr uint32_t kKVBytes = kSpan * 128;
+constexpr uint32_t kStageBytes = kQBytes + 2 * kKVBytes;
+constexpr uint32_t kOffStage = 0;
+constexpr uint32_t kOffOut = kStages * kStageBytes;          // [kOutSlots] staging tiles
+constexpr uint32_t kOffL = kOffOut + kOutSlots * kQBytes;    // float [2][128]
+enum : int {
+  BAR_QK_FULL = 0,                       // [kStages] Q and K landed
+  BAR_V_FULL = BAR_QK_FULL + kStages,    // [kStages]
+  BAR_READY = BAR_V_FULL + kStages,      // [kStages] Q rotated
+  BAR_EMPTY = BAR_READY + kStages,       // [kStages] stage consumed
+  BAR_S_FULL = BAR_EMPTY + kStages,      // [2]
+  BAR_P_FULL = BAR_S_FULL + 2,           // [2]
+  BAR_O_FULL = BAR_P_FULL + 2,           // [2]
+  BAR_O_EMPTY = BAR_O_FULL + 2,          // [2]
+  BAR_L_FULL = BAR_O_EMPTY + 2,          // [2]
+  BAR_L_EMPTY = BAR_L_FULL + 2,          // [2]
+  BAR_MMA_DONE = BAR_L_EMPTY + 2,
+  NUM_BARS
+};
+constexpr uint32_t kOffBar = kOffL + 2 * 128 * 4;
+constexpr uint32_t kOffMisc = kOffBar + NUM_BARS * 8;
+constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+__host__ __device__ constexpr uint32_t tmem_s(int m) { return m ? 160u : 0u; }
+__host__ __device__ constexpr uint32_t tmem_o(int m) { return m ? 384u : 320u; }
+
+struct Ctx {
+  uint32_t sbase;
+  volatile int* abort_flag;
+  int* err;
+  __device__ uint32_t bar(int i) const { return sbase + kOffBar + 8u * static_cast<uint32_t>(i); }
+  __device__ bool wait(int i, uint32_t parity) const {
+    return mbar_wait(bar(i), parity, abort_flag, err, kErrTimeout, kWaitTimeoutNs);
+  }
+  __device__ bool wait_warp(int i, uint32_t parity) const {
+    return mbar_wait_warp(bar(i), parity, abort_flag, err, kErrTimeout, kWaitTimeoutNs);
+  }
+  __device__ uint32_t q(int s) const { return sbase + kOffStage + s * kStageBytes; }
+  __device__ uint32_t k(int s) const { return q(s) + kQBytes; }
+  __device__ uint32_t v(int s) const { return q(s) + kQBytes + kKVBytes; }
+};
+
+struct Item {
+  int b, g, q0;
+};
+
+// The k-th item of CTA `cta` (round-robin over items ordered by token tile,
+// then kv head, then batch); false past the end.
+__device__ __forceinline__ bool item_for(const PrefillArgs& a, int k, int cta, Item* it) {
+  const int idx = k * static_cast<int>(gridDim.x) + cta;
+  if (idx >= a.n_items) return false;
+  const int per_tile = kNumKvHeads * a.batch;
+  it->q0 = (idx / per_tile) * kTokens;
+  const int rem = idx % per_tile;
+  it->g = rem % kNumKvHeads;
+  it->b = rem / kNumKvHeads;
+  return true;
+}
+
+}  // namespace band
+
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_band_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs args) {
+  using namespace band;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  band::Ctx ctx;
+  ctx.sbase = smem_u32(smem);
+  ctx.abort_flag = reinterpret_cast<volatile int*>(smem + band::kOffMisc + 4);
+  ctx.err = args.err;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + band::kOffMisc);
+  float* l_smem = reinterpret_cast<float*>(smem + band::kOffL);
+
+  const int warp = static_cast<int>(threadIdx.x >> 5);
+  const int lane = static_cast<int>(threadIdx.x & 31);
+  const int cta = static_cast<int>(blockIdx.x);
+  const int S = args.seqlen;
+  const int W = args.window;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < band::kStages; ++s) {
+      mbar_init(ctx.bar(band::BAR_QK_FULL + s), 1);
+      mbar_init(ctx.bar(band::BAR_V_FULL + s), 1);
+      mbar_init(ctx.bar(band::BAR_READY + s), 2);
+      mbar_init(ctx.bar(band::BAR_EMPTY + s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(ctx.bar(band::BAR_S_FULL + i), 1);
+      mbar_init(ctx.bar(band::BAR_P_FULL + i), 4);
+      mbar_init(ctx.bar(band::BAR_O_FULL + i), 1);
+      mbar_init(ctx.bar(band::BAR_O_EMPTY + i), 4);
+      mbar_init(ctx.bar(band::BAR_L_FULL + i), 4);
+      mbar_init(ctx.bar(band::BAR_L_EMPTY + i), 4);
+    }
+    mbar_init(ctx.bar(band::BAR_MMA_DONE), 1);
+    *ctx.abort_flag = (*reinterpret_cast<volatile int*>(args.err) & kErrTimeout) ? 1 : 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const bool skip = *ctx.abort_flag != 0;
+  const int wg = warp >> 2;
+
+  if (wg == 0) {
+    setmaxnreg_dec<kRegsLight>();
+    if (warp == 0) {
+      // -------------------------------------------------------------- producer
+      if (lane == 0 && !skip) {
+        prefetch_tensormap(&maps.q);
+        prefetch_tensormap(&maps.k_band);
+        prefetch_tensormap(&maps.v_band);
+        int k = 0;
+        band::Item it;
+        for (; band::item_for(args, k, cta, &it); ++k) {
+          const int s = k % band::kStages;
+          if (k >= band::kStages &&
+              !ctx.wait(band::BAR_EMPTY + s, ((k / band::kStages) - 1) & 1))
+            break;
+          const int kb = it.q0 - 128;
+          mbar_arrive_expect_tx(ctx.bar(band::BAR_QK_FULL + s), band::kQBytes + band::kKVBytes);
+          tma_load_4d(ctx.q(s), &maps.q, ctx.bar(band::BAR_QK_FULL + s), 0, it.g * kGroup, it.q0,
+                      it.b);
+          tma_load_4d(ctx.k(s), &maps.k_band, ctx.bar(band::BAR_QK_FULL + s), 0, it.g, kb, it.b);
+          mbar_arrive_expect_tx(ctx.bar(band::BAR_V_FULL + s), band::kKVBytes);
+          tma_load_4d(ctx.v(s), &maps.v_band, ctx.bar(band::BAR_V_FULL + s), 0, it.g, kb, it.b);
+        }
+        if (*ctx.abort_flag) {
+          volatile int never = 0;
+          for (int i = max(0, k - band::kStages); i < k; ++i) {
+            const int s = i % band::kStages;
+            const uint32_t ph = (i / band::kStages) & 1;
+            mbar_wait(ctx.bar(band::BAR_QK_FULL + s), ph, &never, nullptr, 0, kWaitTimeoutNs);
+            mbar_wait(ctx.bar(band::BAR_V_FULL + s), ph, &never, nullptr, 0, kWaitTimeoutNs);
+          }
+        }
+      }
+    } else if (warp == 1) {
+      // -------------------------------------------------------------- MMA issuer
+      if (lane == 0 && !skip) {
+        constexpr uint32_t idesc_qk = idesc_bf16(128, band::kSpan, false);
+        constexpr uint32_t idesc_pv = idesc_bf16(128, kHeadDim, true);
+        auto do_pv = [&](int p) -> bool {
+          const int m = p & 1, s = p % band::kStages;
+          if (!ctx.wait(band::BAR_V_FULL + s, (p / band::kStages) & 1)) return false;
+          if (!ctx.wait(band::BAR_P_FULL + m, (p >> 1) & 1)) return false;
+          if (p >= 2 && !ctx.wait(band::BAR_O_EMPTY + m, ((p >> 1) - 1) & 1)) return false;
+          tc_fence_after_sync();
+#pragma unroll
+          for (int kk = 0; kk < band::kSpan / 16; ++kk)
+            mma_bf16_ts(tmem + band::tmem_o(m), tmem + band::tmem_s(m) + 8 * kk,
+                        sdesc_sw128(ctx.v(s) + 2048 * kk), idesc_pv, kk > 0 ? 1u : 0u);
+          mma_commit(ctx.bar(band::BAR_O_FULL + m));
+          mma_commit(ctx.bar(band::BAR_EMPTY + s));
+          return true;
+        };
+        int k = 0;
+        band::Item it;
+        bool ok = true;
+        for (; band::item_for(args, k, cta, &it); ++k) {
+          const int m = k & 1, s = k % band::kStages;
+          if (!(ok = ctx.wait(band::BAR_QK_FULL + s, (k / band::kStages) & 1) &&
+                     ctx.wait(band::BAR_READY + s, (k / band::kStages) & 1)))
+            break;
+          tc_fence_after_sync();
+#pragma unroll
+          for (int kk = 0; kk < kHeadDim / 16; ++kk)
+            mma_bf16_ss(tmem + band::tmem_s(m), sdesc_sw128(ctx.q(s) + 32 * kk),
+                        sdesc_sw128(ctx.k(s) + 32 * kk), idesc_qk, kk > 0 ? 1u : 0u);
+          mma_commit(ctx.bar(band::BAR_S_FULL + m));
+          if (k > 0 && !(ok = do_pv(k - 1))) break;
+        }
+        if (ok && k > 0) do_pv(k - 1);
+        mma_commit(ctx.bar(band::BAR_MMA_DONE));
+        volatile int never = 0;
+        mbar_wait(ctx.bar(band::BAR_MMA_DONE), 0, &never, nullptr, 0, kWaitTimeoutNs);
+      }
+    } else {
+      // -------------------------------------------------------------- RoPE
+      const int t = static_cast<int>(threadIdx.x) - 64;  // 0..63
+      band::Item it;
+      bool ok = !skip;
+      for (int k = 0; ok && band::item_for(args, k, cta, &it); ++k) {
+        const int s = k % band::kStages;
+        int pq[2];
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int tok = it.q0 + ((t + 64 * rr) >> 3);
+          pq[rr] = tok < S ? load_position(args, it.b, tok) : -1;
+        }
+        if (!(ok = ctx.wait_warp(band::BAR_QK_FULL + s, (k / band::kStages) & 1))) break;
+        uint8_t* qt = smem + band::kOffStage + s * band::kStageBytes;
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr)
+          if (pq[rr] >= 0)
+            rope_row(qt + (t + 64 * rr) * 128, t + 64 * rr,
+                     args.rope + static_cast<size_t>(pq[rr]) * kRopePairs);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ctx.bar(band::BAR_READY + s));
+      }
+    }
+  } else if (wg == 1 || wg == 2) {
+    // ---------------------------------------------------------------- softmax
+    setmaxnreg_inc<kRegsSoftmax>();
+    const int m = wg - 1;
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + band::tmem_s(m);
+    band::Item it;
+    bool ok = !skip;
+    for (int k = m, i = 0; ok && band::item_for(args, k, cta, &it); k += 2, ++i) {
+      // row token q0 + d sees keys (q0+d-W, q0+d], i.e. span columns
+      // [max(128-q0, d+129-W), d+128] of the span starting at key q0-128
+      const int d = r >> 3;
+      const int c_lo = max(128 - it.q0, d + 129 - W);
+      const int c_hi = d + 128;
+      const float sink = __ldg(args.sinks + it.g * kGroup + (r & 7));
+      const bool sink_off = isinf(sink) && sink < 0.f;
+      if (!(ok = ctx.wait_warp(band::BAR_S_FULL + m, i & 1))) break;
+      tc_fence_after_sync();
+      uint32_t sv[band::kSpan];
+      tmem_ld144_split(tS, sv);
+      float mx = sink_off ? -INFINITY : sink * kLog2e;
+#pragma unroll
+      for (int c = 0; c < band::kSpan; ++c) {
+        const float x = (c >= c_lo && c <= c_hi) ? __uint_as_float(sv[c]) * kScaleLog2 : -INFINITY;
+        sv[c] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
+      }
+      const float mr = mx == -INFINITY ? 0.f : mx;
+      float l0 = sink_off ? 0.f : ex2_approx(sink * kLog2e - mr), l1 = 0.f;
+      // probabilities packed to bf16 in place: sv[c] <- (p[2c], p[2c+1])
+#pragma unroll
+      for (int c = 0; c < band::kSpan / 2; ++c) {
+        const float p0 = ex2_approx(__uint_as_float(sv[2 * c]) - mr);
+        const float p1 = ex2_approx(__uint_as_float(sv[2 * c + 1]) - mr);
+        l0 += p0;
+        l1 += p1;
+        sv[c] = pack_bf16x2(p0, p1);
+      }
+      {
+        uint32_t a[64], b8[8];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) a[c] = sv[c];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) b8[c] = sv[64 + c];
+        tmem_st64(tS, a);
+        tmem_st8(tS + 64, b8);
+      }
       tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ctx.bar(BAR_P_FULL + m));
+      if (lane == 0) mbar_arrive(ctx.bar(band::BAR_P_FULL + m));
+      if (i >= 1 && !(ok = ctx.wait_warp(band::BAR_L_EMPTY + m, (i - 1) & 1))) break;
+      l_smem[m * 128 + r] = l0 + l1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ctx.bar(band::BAR_L_FULL + m));
     }
-    // epilogue: O / l -> bf16 -> (swizzled) staging in the Q tile -> TMA store
-    uint8_t* stage = smem + kOffQ + m * kTileBytes;
-    if (ok && ctx.wait(BAR_O_FULL + m, 0)) {
-      tc_fence_after_sync();
-      const float inv_l = 1.f / l;
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    setmaxnreg_dec<kRegsLight>();
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    band::Item it;
+    for (int k = 0; band::item_for(args, k, cta, &it); ++k) {
+      const int m = k & 1, i = k >> 1;
+      uint8_t* stage = smem + band::kOffOut + (k % band::kOutSlots) * band::kQBytes;
+      bool ok = !skip && !*ctx.abort_flag && ctx.wait_warp(band::BAR_O_FULL + m, i & 1);
+      uint32_t ov[64];
+      if (ok) {
+        tc_fence_after_sync();
+        tmem_ld64(tmem + lane_off + band::tmem_o(m), ov);
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ctx.bar(band::BAR_O_EMPTY + m));
+      }
+      ok = ok && ctx.wait_warp(band::BAR_L_FULL + m, i & 1);
+      if (ok) {
+        const float l = l_smem[m * 128 + r];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ctx.bar(band::BAR_L_EMPTY + m));
+        const float inv_l = 1.f / l;
 #pragma unroll
-      for (int ch = 0; ch < kHeadDim / 32; ++ch) {
-        uint32_t ov[32];
-        tmem_ld32(tO + ch * 32, ov);
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 8; ++cc) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             w[e] = pack_bf16x2(__uint_as_float(ov[8 * cc + 2 * e]) * inv_l,
                                __uint_as_float(ov[8 * cc + 2 * e + 1]) * inv_l);
-          const int chunk = ch * 4 + cc;
-          *reinterpret_cast<uint4*>(stage + r * 128 + ((chunk ^ (r & 7)) << 4)) =
+          *reinterpret_cast<uint4*>(stage + r * 128 + ((cc ^ (r & 7)) << 4)) =
               make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       fence_async_smem();
-    }
-    named_barrier(1 + m, 128);
-    if (r == 0 && !skip && !*ctx.abort_flag && q0 + m * kTokensPerM < S) {
-      tma_store_4d(&maps.o, ctx.sbase + kOffQ + m * kTileBytes, 0, g * kGroup,
-                   q0 + m * kTokensPerM, b);
-      tma_store_commit();
-      tma_store_wait_all();
-    }
-  } else if (warp >= 12) {
-    // ---------------------------------------------------------------- RoPE
-    const int t = static_cast<int>(threadIdx.x) - 384;  // 0..127
-    bool ok = !skip && ctx.wait(BAR_Q_FULL, 0);
-    if (ok) {
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const int tok = q0 + m * kTokensPerM + (t >> 3);
-        if (tok < S)
-          rope_row(smem + kOffQ + m * kTileBytes + t * 128, t,
-                   args.rope + static_cast<size_t>(load_position(args, b, tok)) * kRopePairs);
+      // At most two stores (items k-1, k-2) may still be reading staging, so
+      // the slot of item k-3, which item k+1 reuses, is free after the barrier.
+      if (threadIdx.x == 384) tma_store_wait_read_pending<band::kOutSlots - 2>();
+      named_barrier(1, 128);
+      if (threadIdx.x == 384) {
+        if (ok && !*ctx.abort_flag && it.q0 < S)
+          tma_store_4d(&maps.o, smem_u32(stage), 0, it.g * kGroup, it.q0, it.b);
+        tma_store_commit();
       }
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ctx.bar(BAR_Q_READY));
     }
-    for (int it = 0; ok && it < n_tiles; ++it) {
-      const int s = it % kStages;
-      if (!(ok = ctx.wait(BAR_K_FULL + s, (it / kStages) & 1))) break;
-      const int key = (jt0 + it) * kBlockN + t;
-      if (key < S)
-        rope_row(smem + kOffK + s * kTileBytes + t * 128, t,
-                 args.rope + static_cast<size_t>(load_position(args, b, key)) * kRopePairs);
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ctx.bar(BAR_K_READY + s));
-    }
+    if (threadIdx.x == 384) tma_store_wait_all();
   }
 
   tc_fence_before_sync();
@@ -431,12 +886,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+bool prefill_uses_band(int window) { return window > 0 && window <= 128; }
+
+int prefill_items(int batch, int seqlen, int window) {
+  const int tokens = prefill_uses_band(window) ? band::kTokens : kBlockQ;
+  return (seqlen + tokens - 1) / tokens * kNumKvHeads * batch;
+}
+
 cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream) {
+  const int grid = args.n_items < args.grid ? args.n_items : args.grid;
+  if (prefill_uses_band(args.window)) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_band_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(band::kSmemBytes));
+    if (e != cudaSuccess) return e;
+    prefill_band_kernel<<<grid, kThreads, band::kSmemBytes, stream>>>(maps, args);
+    return cudaGetLastError();
+  }
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(args.n_qtiles), kNumKvHeads,
-                  static_cast<unsigned>(args.batch));
   prefill_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps, args);
   return cudaGetLastError();
 }

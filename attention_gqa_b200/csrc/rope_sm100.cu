@@ -1,0 +1,88 @@
+// Rotary embedding (half-split RoPE of the gpt-oss pages: inteligile
+// techniques map rows "Partial RoPE" and "Layers without positional encoding
+// (NoPE)"; rope_theta = 150000 in the llm-atlas field table).
+//
+// rope_table_kernel: for every position p < 131072 and pair k < 32 the
+//   (cos, sin) of p * theta^(-2k/64). Angles reach 1.3e5 rad, so they are
+//   formed and reduced in fp64; only the results are stored as fp32.
+// rope_keys_kernel: rotates every key row once per layer into a workspace,
+//   so the attention kernels, which read each key tile many times, never
+//   rotate keys. HBM bound: 128 bytes read and written per row.
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace gqa {
+namespace {
+
+__global__ void rope_table_kernel(float2* __restrict__ table) {
+  const int idx = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
+  if (idx >= kMaxPosition * kRopePairs) return;
+  const int p = idx / kRopePairs;
+  const int k = idx % kRopePairs;
+  const double inv_freq = pow(kRopeTheta, -2.0 * static_cast<double>(k) / kHeadDim);
+  double s, c;
+  sincos(static_cast<double>(p) * inv_freq, &s, &c);
+  table[idx] = make_float2(static_cast<float>(c), static_cast<float>(s));
+}
+
+// Four threads per 64-element row; thread c rotates the 16-byte chunks c and
+// c+4 (elements 8c..8c+7 pair with 8c+32..8c+39). Rows are [token][kv head],
+// so the eight rows of a token share one position and one table row.
+__global__ void __launch_bounds__(256) rope_keys_kernel(const uint4* __restrict__ k,
+                                                        const int32_t* __restrict__ pos,
+                                                        const float2* __restrict__ table,
+                                                        uint4* __restrict__ k_rot,
+                                                        int64_t n_rows, int* err) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+       idx < n_rows * 4; idx += stride) {
+    const int64_t row = idx >> 2;
+    const int c = static_cast<int>(idx & 3);
+    int p = __ldg(pos + (row >> 3));
+    if (p < 0 || p >= kMaxPosition) {
+      atomicOr(err, kErrPosition);
+      p = p < 0 ? 0 : kMaxPosition - 1;
+    }
+    const uint4 a = __ldg(k + row * 8 + c);
+    const uint4 h = __ldg(k + row * 8 + c + 4);
+    const float4* t4 = reinterpret_cast<const float4*>(table + static_cast<int64_t>(p) * kRopePairs +
+                                                       8 * c);
+    const float4 t0 = __ldg(t4 + 0), t1 = __ldg(t4 + 1), t2 = __ldg(t4 + 2), t3 = __ldg(t4 + 3);
+    const float cv[8] = {t0.x, t0.z, t1.x, t1.z, t2.x, t2.z, t3.x, t3.z};
+    const float sv[8] = {t0.y, t0.w, t1.y, t1.w, t2.y, t2.w, t3.y, t3.w};
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+    const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+    uint32_t ya[4], yh[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x1l = bf16lo_to_f32(aw[e]), x1h = bf16hi_to_f32(aw[e]);
+      const float x2l = bf16lo_to_f32(hw[e]), x2h = bf16hi_to_f32(hw[e]);
+      const float cl = cv[2 * e], ch = cv[2 * e + 1], sl = sv[2 * e], sh = sv[2 * e + 1];
+      ya[e] = pack_bf16x2(fmaf(x1l, cl, -x2l * sl), fmaf(x1h, ch, -x2h * sh));
+      yh[e] = pack_bf16x2(fmaf(x2l, cl, x1l * sl), fmaf(x2h, ch, x1h * sh));
+    }
+    k_rot[row * 8 + c] = make_uint4(ya[0], ya[1], ya[2], ya[3]);
+    k_rot[row * 8 + c + 4] = make_uint4(yh[0], yh[1], yh[2], yh[3]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_rope_table(float2* table, cudaStream_t stream) {
+  const int n = kMaxPosition * kRopePairs;
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, stream>>>(table);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_keys(const void* k, const int32_t* pos, const float2* table, void* k_rot,
+                             int64_t n_tokens, int grid_cap, int* err, cudaStream_t stream) {
+  const int64_t n_rows = n_tokens * kNumKvHeads;
+  const int64_t threads = n_rows * 4;
+  int64_t blocks = (threads + 255) / 256;
+  if (blocks > grid_cap) blocks = grid_cap;
+  rope_keys_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      static_cast<const uint4*>(k), pos, table, static_cast<uint4*>(k_rot), n_rows, err);
+  return cudaGetLastError();
+}
+
+}  // namespace gqa

@@ -245,7 +245,9 @@ def run_ours(args, rank: int, world: int):
                         sinks=torch.from_numpy(x["sinks"]).to(dev),
                         pos=torch.from_numpy(x["pos"]).to(dev), window=window,
                         out=torch.empty(PREFILL_B, PREFILL_S, NQ, D, dtype=torch.bfloat16,
-                                        device=dev), host=x))
+                                        device=dev),
+                        ws=torch.empty(gqa.prefill_workspace_bytes(PREFILL_B, PREFILL_S),
+                                       dtype=torch.uint8, device=dev), host=x))
     dec = []
     for layer, window in DECODE_LAYERS:
         x = synth.make_decode_inputs(4, layer, DECODE_B, DECODE_L)
@@ -262,7 +264,8 @@ def run_ours(args, rank: int, world: int):
         if ev is not None:
             ev[i].record(stream)
         for p in pre:
-            gqa.prefill(p["q"], p["k"], p["v"], p["sinks"], p["pos"], p["window"], out=p["out"])
+            gqa.prefill(p["q"], p["k"], p["v"], p["sinks"], p["pos"], p["window"], out=p["out"],
+                        workspace=p["ws"])
             i += 1
             if ev is not None:
                 ev[i].record(stream)
@@ -370,7 +373,8 @@ def run_ours(args, rank: int, world: int):
                        "parallelism": "dp%d (independent replicas)" % world,
                        "prefill_ms_per_step": pre_ms, "decode_ms_per_step": dec_ms,
                        "wall_s": t_wall},
-            "roofline": {"kernel": "prefill_kernel (full-causal layer, S=4096)", "bound": "tensor",
+            "roofline": {"kernel": "prefill (key rotation + prefill_kernel, full-causal layer, "
+                                   "S=4096)", "bound": "tensor",
                          "achieved": full_tf, "peak": tf_burst, "unit": "TFLOP/s",
                          "frac": full_tf / tf_burst, "peak_source": peak_src + " (burst)",
                          "traffic": traffic,
@@ -382,7 +386,8 @@ def run_ours(args, rank: int, world: int):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "what": "prefill layers via host buffers"},
-            "gpu_launches": args.steps * (len(PREFILL_LAYERS) + 2 * len(DECODE_LAYERS)),
+            # per step: key rotation + attention per prefill layer, split-KV + combine per decode
+            "gpu_launches": args.steps * (2 * len(PREFILL_LAYERS) + 2 * len(DECODE_LAYERS)),
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -95,6 +95,12 @@ int gptoss_attn_init(void);
 int gptoss_attn_rope_table(const void** table);
 
 /*
+ * Bytes of device workspace gptoss_attn_prefill() needs: room for the rotated
+ * keys, batch * seqlen * 8 * 64 bf16 values. Returns 0 for invalid sizes.
+ */
+size_t gptoss_attn_prefill_workspace_bytes(int batch, int seqlen);
+
+/*
  * Prefill: causal grouped-query attention over whole sequences.
  *   q      bf16 [batch][seqlen][64][64]   (token-major, as the projections emit)
  *   k, v   bf16 [batch][seqlen][8][64]
@@ -104,11 +110,18 @@ int gptoss_attn_rope_table(const void** table);
  *   window <= 0: full causal; W > 0: key j visible to query i iff i-W < j <= i
  *   out    bf16 [batch][seqlen][64][64]; must not overlap the inputs
  *   batch >= 1, 1 <= seqlen <= 131072 (batch * seqlen * 8 KB must fit the device)
- * q and k are rotated inside the kernel; k and v are read as given.
+ *   workspace, workspace_bytes: caller-owned device scratch of at least
+ *          gptoss_attn_prefill_workspace_bytes(batch, seqlen) bytes, 16-byte
+ *          aligned, not overlapping the other tensors; it receives the rotated
+ *          keys (each key is rotated once per call, not once per query tile)
+ *          and is garbage afterwards. Calls that overlap in time need
+ *          separate workspaces.
+ * Two kernels run on `stream`: the key rotation, then the attention, which
+ * rotates the query rows itself; v is read as given.
  */
 int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float* sinks,
                         const int32_t* pos, int window, void* out, int batch, int seqlen,
-                        cudaStream_t stream);
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Bytes of device workspace gptoss_attn_decode() needs for these sizes.

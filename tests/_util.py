@@ -33,3 +33,24 @@ def compare(got: np.ndarray, ref: np.ndarray, what: str = ""):
     assert mx <= MAX_ABS_TOL, "%s: max abs err %.3e at %s (tol %.1e)" % (what, mx, where, MAX_ABS_TOL)
     assert mean <= MEAN_ABS_TOL, "%s: mean abs err %.3e (tol %.1e)" % (what, mean, MEAN_ABS_TOL)
     return mx, mean, where
+
+
+# Bound for stress inputs whose softmax is nearly one-hot, so the output is
+# close to a single V row of magnitude up to ~5. Rounding each probability to
+# bf16 (8 significant bits) moves the weighted sum by up to 2^-9 * sum p|v|/l,
+# at most ~1e-2 for |v| <= 5, covered by the 2e-2 absolute term; rounding the
+# output itself costs up to 2^-8 |out| on top.
+STRESS_ATOL = 2e-2
+STRESS_RTOL = 2.0 ** -8
+
+
+def compare_rel(got: np.ndarray, ref: np.ndarray, what: str = "", atol: float = STRESS_ATOL,
+                rtol: float = STRESS_RTOL):
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), "%s: non-finite output" % what
+    err = np.abs(got - ref)
+    bound = atol + rtol * np.abs(ref)
+    worst = np.unravel_index(int(np.argmax(err - bound)), err.shape)
+    assert np.all(err <= bound), "%s: err %.3e > bound %.3e at %s (ref %.4f)" % (
+        what, err[worst], bound[worst], worst, ref[worst])
+    return float(err.max())

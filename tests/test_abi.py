@@ -50,8 +50,12 @@ def test_abi_version_and_status_strings(lib):
     assert lib.gptoss_attn_status_string(12345).decode() == "unknown status"
 
 
-def _prefill(lib, q=16, k=32, v=48, sinks=64, pos=80, window=0, out=96, batch=1, seqlen=8):
-    return lib.gptoss_attn_prefill(q, k, v, sinks, pos, window, out, batch, seqlen, None)
+def _prefill(lib, q=16, k=32, v=48, sinks=64, pos=80, window=0, out=96, batch=1, seqlen=8,
+             ws=112, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = max(1, lib.gptoss_attn_prefill_workspace_bytes(batch, seqlen))
+    return lib.gptoss_attn_prefill(q, k, v, sinks, pos, window, out, batch, seqlen, ws, ws_bytes,
+                                   None)
 
 
 def test_prefill_argument_errors(lib):
@@ -63,6 +67,13 @@ def test_prefill_argument_errors(lib):
     assert _prefill(lib, seqlen=131073) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
     assert _prefill(lib, k=40) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
     assert _prefill(lib, pos=82) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
+    assert _prefill(lib, ws=None) == c["GPTOSS_ATTN_ERR_NULL_PTR"]
+    assert _prefill(lib, ws=120) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
+    need = lib.gptoss_attn_prefill_workspace_bytes(2, 100)
+    assert need == 2 * 100 * 8 * 64 * 2
+    assert _prefill(lib, batch=2, seqlen=100, ws_bytes=need - 1) == \
+        c["GPTOSS_ATTN_ERR_SMALL_WORKSPACE"]
+    assert lib.gptoss_attn_prefill_workspace_bytes(0, 5) == 0
 
 
 def _decode(lib, q=16, kc=32, vc=48, sinks=64, ln=80, window=0, out=96, batch=2, max_len=100,
