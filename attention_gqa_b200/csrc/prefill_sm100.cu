@@ -23,9 +23,10 @@
 //                 one 128-column TMEM load per tile, sink-seeded online softmax
 //                 in log2 units, bf16 P written back over S.
 //   WG3           epilogue: O / l -> bf16 -> swizzled staging -> TMA store.
-// TMEM (512 columns): S0 [0,128), S1 [128,256) with P aliased on their first
-// 64 columns; O[m][item parity] at 256 + 64*(2*parity + m), so the next
-// item's P.V never waits for the previous item's epilogue.
+// TMEM (512 columns): S0 [0,128), S1 [128,256), P0 [256,320), P1 [320,384),
+// O0 [384,448), O1 [448,512). The softmax releases S right after loading it,
+// so Q K^T of tile j+1 overlaps the softmax of tile j and P.V of tile j
+// overlaps the softmax of tile j+1.
 // The running max starts at sigma*log2(e) with l = 1; O is rescaled only when
 // the max grows by more than 2^8 (exact: O and l share the reference).
 #include <cmath>
@@ -44,14 +45,17 @@ constexpr int kThreads = 512;
 constexpr uint32_t kTileBytes = 128 * 128;  // 128 rows of 64 bf16
 
 constexpr uint32_t kTmemCols = 512;
-__host__ __device__ constexpr uint32_t tmem_s(int m) { return m ? 128u : 0u; }
-__host__ __device__ constexpr uint32_t tmem_o(int m, int ob) {
-  return 256u + 64u * static_cast<uint32_t>(2 * ob + m);
-}
+// TMEM columns of M tile m: S (fp32, 128 columns), P (bf16 pairs, 64 columns)
+// and the O accumulator (fp32, 64 columns). P has columns of its own, so the
+// next tile's S = Q K^T can be computed while the softmax still works on the
+// current one.
+__host__ __device__ constexpr uint32_t tmem_s(int m) { return 128u * static_cast<uint32_t>(m); }
+__host__ __device__ constexpr uint32_t tmem_p(int m) { return 256u + 64u * static_cast<uint32_t>(m); }
+__host__ __device__ constexpr uint32_t tmem_o(int m) { return 384u + 64u * static_cast<uint32_t>(m); }
 
 // Register budgets after the warpgroup split; launch is 512 x 128.
-constexpr uint32_t kRegsLight = 88;     // WG0 and WG3
-constexpr uint32_t kRegsSoftmax = 168;  // WG1 and WG2
+constexpr uint32_t kRegsLight = 72;     // WG0 and WG3
+constexpr uint32_t kRegsSoftmax = 184;  // WG1 and WG2
 static_assert(2 * 128 * kRegsLight + 2 * 128 * kRegsSoftmax <= 512 * 128, "register split");
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -65,13 +69,16 @@ enum : int {
   BAR_K_FULL = BAR_Q_EMPTY + 2,          // [kStages]
   BAR_V_FULL = BAR_K_FULL + kStages,     // [kStages]
   BAR_KV_EMPTY = BAR_V_FULL + kStages,   // [kStages]
-  BAR_S_FULL = BAR_KV_EMPTY + kStages,   // [2] per M tile
-  BAR_P_FULL = BAR_S_FULL + 2,           // [2]
-  BAR_O_FULL = BAR_P_FULL + 2,           // [4] m*2 + parity
-  BAR_O_EMPTY = BAR_O_FULL + 4,          // [4]
-  BAR_L_FULL = BAR_O_EMPTY + 4,          // [2]
+  BAR_S_FULL = BAR_KV_EMPTY + kStages,   // [2] per M tile: S written
+  BAR_S_FREE = BAR_S_FULL + 2,           // [2] S read by the softmax
+  BAR_P_FULL = BAR_S_FREE + 2,           // [2] P written
+  BAR_P_FREE = BAR_P_FULL + 2,           // [2] P.V done (P and O free)
+  BAR_O_FULL = BAR_P_FREE + 2,           // [2] item's O complete
+  BAR_O_EMPTY = BAR_O_FULL + 2,          // [2] item's O read by the epilogue
+  BAR_L_FULL = BAR_O_EMPTY + 2,          // [2]
   BAR_L_EMPTY = BAR_L_FULL + 2,          // [2]
-  BAR_MMA_DONE = BAR_L_EMPTY + 2,
+  BAR_TURN = BAR_L_EMPTY + 2,            // [2] exp-loop turn of softmax warpgroup m
+  BAR_MMA_DONE = BAR_TURN + 2,
   NUM_BARS
 };
 
@@ -79,7 +86,9 @@ constexpr uint32_t kOffQ = 0;  // [2 slots][2 halves] tiles
 constexpr uint32_t kOffK = kOffQ + 4 * kTileBytes;
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
 constexpr uint32_t kOffL = kOffV + kStages * kTileBytes;  // float [2][128]
-constexpr uint32_t kOffBar = kOffL + 2 * 128 * 4;
+constexpr uint32_t kOffTab = kOffL + 2 * 128 * 4;  // float2 [2 slots][32 tokens][32]
+constexpr uint32_t kTabSlotBytes = kBlockQ * kRopePairs * 8;
+constexpr uint32_t kOffBar = kOffTab + 2 * kTabSlotBytes;
 constexpr uint32_t kOffMisc = kOffBar + NUM_BARS * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
 
@@ -122,24 +131,17 @@ __device__ __forceinline__ bool item_for(const PrefillArgs& a, int k, int cta, I
   return true;
 }
 
-__device__ __forceinline__ int load_position(const PrefillArgs& a, int b, int t) {
-  int p = __ldg(a.pos + static_cast<size_t>(b) * a.seqlen + t);
-  if (p < 0 || p >= kMaxPosition) {
-    atomicOr(a.err, kErrPosition);
-    p = p < 0 ? 0 : kMaxPosition - 1;
-  }
-  return p;
-}
-
 // Rotate one 64-element row stored at `row` (128 bytes, 128B-swizzled with
-// row index r) by the table entry `cs` of its position, in place.
-__device__ __forceinline__ void rope_row(uint8_t* row, int r, const float2* __restrict__ cs) {
+// row index r) by the (cos, sin) table row `cs` of its position, in place.
+// Both live in shared memory: the producer stages the table rows an item
+// needs (one per token) next to its Q tile.
+__device__ __forceinline__ void rope_row(uint8_t* row, int r, const float2* cs) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     uint4* plo = reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4));
     uint4* phi = reinterpret_cast<uint4*>(row + (((c + 4) ^ (r & 7)) << 4));
     const float4* t4 = reinterpret_cast<const float4*>(cs + 8 * c);
-    const float4 t0 = __ldg(t4 + 0), t1 = __ldg(t4 + 1), t2 = __ldg(t4 + 2), t3 = __ldg(t4 + 3);
+    const float4 t0 = t4[0], t1 = t4[1], t2 = t4[2], t3 = t4[3];
     const uint4 a = *plo, h = *phi;
     const float cv[8] = {t0.x, t0.z, t1.x, t1.z, t2.x, t2.z, t3.x, t3.z};
     const float sv[8] = {t0.y, t0.w, t1.y, t1.w, t2.y, t2.w, t3.y, t3.w};
@@ -159,8 +161,76 @@ __device__ __forceinline__ void rope_row(uint8_t* row, int r, const float2* __re
   }
 }
 
+// Stages the rotary-table rows of tokens q0 .. q0+n-1 of sequence b (one
+// 256-byte row each; the 8 heads of a token share its position) into
+// shared memory at `dst`, completing on `bar`. Returns the bytes requested;
+// tokens past the sequence end are skipped. Run by one thread.
+template <int kTokensPerItem>
+__device__ __forceinline__ uint32_t stage_rope_rows(const PrefillArgs& a, int b, int q0,
+                                                    uint32_t dst, uint32_t bar) {
+  constexpr uint32_t kRowBytes = kRopePairs * sizeof(float2);
+  constexpr int kGroupTok = 8;  // positions loaded together, then their copies issued
+  uint32_t bytes = 0;
+#pragma unroll 1
+  for (int t0 = 0; t0 < kTokensPerItem && q0 + t0 < a.seqlen; t0 += kGroupTok) {
+    int p[kGroupTok];
+#pragma unroll
+    for (int t = 0; t < kGroupTok; ++t)
+      p[t] = q0 + t0 + t < a.seqlen
+                 ? __ldg(a.pos + static_cast<size_t>(b) * a.seqlen + q0 + t0 + t) : 0;
+#pragma unroll
+    for (int t = 0; t < kGroupTok; ++t) {
+      if (q0 + t0 + t >= a.seqlen) break;
+      int pt = p[t];
+      if (pt < 0 || pt >= kMaxPosition) {
+        atomicOr(a.err, kErrPosition);
+        pt = pt < 0 ? 0 : kMaxPosition - 1;
+      }
+      bulk_load(dst + (t0 + t) * kRowBytes, a.rope + static_cast<size_t>(pt) * kRopePairs,
+                kRowBytes, bar);
+      bytes += kRowBytes;
+    }
+  }
+  return bytes;
+}
+
 __device__ __forceinline__ bool key_visible(int kj, int tq, int W) {
   return kj <= tq && (W <= 0 || kj > tq - W);
+}
+
+// S_m = Q_m K^T for one K/V tile (4 MMAs of K = 16 over head_dim 64).
+__device__ __forceinline__ void issue_qk(const Ctx& ctx, uint32_t tmem, int m, int qs, int s) {
+  constexpr uint32_t idesc = idesc_bf16(128, kBlockN, false);
+  const uint32_t qa = ctx.q_tile(qs, m);
+  const uint32_t ka = ctx.sbase + kOffK + s * kTileBytes;
+#pragma unroll
+  for (int kk = 0; kk < kHeadDim / 16; ++kk)
+    mma_bf16_ss(tmem + tmem_s(m), sdesc_sw128(qa + 32 * kk), sdesc_sw128(ka + 32 * kk), idesc,
+                kk > 0 ? 1u : 0u);
+}
+
+// O_m (+)= P_m V for both M tiles of global tile G (item n), then the commits
+// that release P, the K/V stage and, after an item's last tile, O.
+__device__ __forceinline__ bool issue_pv_tile(const Ctx& ctx, uint32_t tmem, int G, int n,
+                                              bool first, bool last) {
+  constexpr uint32_t idesc = idesc_bf16(128, kHeadDim, true);
+  const int s = G % kStages;
+  if (!ctx.wait(BAR_V_FULL + s, (G / kStages) & 1)) return false;
+  const uint32_t va = ctx.sbase + kOffV + s * kTileBytes;
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    if (!ctx.wait(BAR_P_FULL + m, G & 1)) return false;
+    if (first && n >= 1 && !ctx.wait(BAR_O_EMPTY + m, (n - 1) & 1)) return false;
+    tc_fence_after_sync();
+#pragma unroll
+    for (int kk = 0; kk < kBlockN / 16; ++kk)
+      mma_bf16_ts(tmem + tmem_o(m), tmem + tmem_p(m) + 8 * kk, sdesc_sw128(va + 2048 * kk), idesc,
+                  (!first || kk > 0) ? 1u : 0u);
+    mma_commit(ctx.bar(BAR_P_FREE + m));
+    if (last) mma_commit(ctx.bar(BAR_O_FULL + m));
+  }
+  mma_commit(ctx.bar(BAR_KV_EMPTY + s));
+  return true;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -187,18 +257,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(ctx.bar(BAR_Q_READY + i), 2);
       mbar_init(ctx.bar(BAR_Q_EMPTY + i), 1);
       mbar_init(ctx.bar(BAR_S_FULL + i), 1);
+      mbar_init(ctx.bar(BAR_S_FREE + i), 4);
       mbar_init(ctx.bar(BAR_P_FULL + i), 4);
+      mbar_init(ctx.bar(BAR_P_FREE + i), 1);
+      mbar_init(ctx.bar(BAR_O_FULL + i), 1);
+      mbar_init(ctx.bar(BAR_O_EMPTY + i), 4);
       mbar_init(ctx.bar(BAR_L_FULL + i), 4);
       mbar_init(ctx.bar(BAR_L_EMPTY + i), 4);
+      mbar_init(ctx.bar(BAR_TURN + i), 4);
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(ctx.bar(BAR_K_FULL + s), 1);
       mbar_init(ctx.bar(BAR_V_FULL + s), 1);
       mbar_init(ctx.bar(BAR_KV_EMPTY + s), 1);
-    }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(ctx.bar(BAR_O_FULL + i), 1);
-      mbar_init(ctx.bar(BAR_O_EMPTY + i), 4);
     }
     mbar_init(ctx.bar(BAR_MMA_DONE), 1);
     // A pipeline timeout earlier left the error word set: skip the work.
@@ -230,11 +301,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (; ok && item_for(args, n, cta, &it); ++n) {
           const int qs = n & 1;
           if (n >= 2 && !(ok = ctx.wait(BAR_Q_EMPTY + qs, ((n >> 1) - 1) & 1))) break;
-          mbar_arrive_expect_tx(ctx.bar(BAR_Q_FULL + qs), 2 * kTileBytes);
+          const uint32_t tab_bytes = kRopePairs * 8 * static_cast<uint32_t>(min(kBlockQ, S - it.q0));
+          mbar_arrive_expect_tx(ctx.bar(BAR_Q_FULL + qs), 2 * kTileBytes + tab_bytes);
           tma_load_4d(ctx.q_tile(qs, 0), &maps.q, ctx.bar(BAR_Q_FULL + qs), 0, it.g * kGroup,
                       it.q0, it.b);
           tma_load_4d(ctx.q_tile(qs, 1), &maps.q, ctx.bar(BAR_Q_FULL + qs), 0, it.g * kGroup,
                       it.q0 + kTokensPerM, it.b);
+          stage_rope_rows<kBlockQ>(args, it.b, it.q0, ctx.sbase + kOffTab + qs * kTabSlotBytes,
+                                   ctx.bar(BAR_Q_FULL + qs));
           nq = n + 1;
           for (int j = 0; j < it.n_tiles; ++j) {
             const int s = G % kStages;
@@ -267,40 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       // -------------------------------------------------------------- MMA issuer
       if (lane == 0 && !skip) {
-        constexpr uint32_t idesc_qk = idesc_bf16(128, kBlockN, false);
-        constexpr uint32_t idesc_pv = idesc_bf16(128, kHeadDim, true);
-        auto issue_qk = [&](int m, int qs, int s) {
-          const uint32_t qa = ctx.q_tile(qs, m);
-          const uint32_t ka = ctx.sbase + kOffK + s * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < kHeadDim / 16; ++kk)
-            mma_bf16_ss(tmem + tmem_s(m), sdesc_sw128(qa + 32 * kk), sdesc_sw128(ka + 32 * kk),
-                        idesc_qk, kk > 0 ? 1u : 0u);
-        };
-        auto issue_pv = [&](int m, int s, int ob, bool accumulate) {
-          const uint32_t va = ctx.sbase + kOffV + s * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < kBlockN / 16; ++kk)
-            mma_bf16_ts(tmem + tmem_o(m, ob), tmem + tmem_s(m) + 8 * kk,
-                        sdesc_sw128(va + 2048 * kk), idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
-        };
-        // The P.V of the previous tile (global index pv_G, item pv_n) is issued
-        // interleaved with the current tile's Q.K^T on the other M tile.
+        // P.V of tile pv_G (item pv_n) is issued after the next tile's Q.K^T:
+        // the softmax releases S as soon as it has loaded it, long before P.
         int pv_G = -1, pv_n = 0;
         bool pv_first = false, pv_last = false;
-        auto do_pv = [&](int m) -> bool {
-          const int s = pv_G % kStages;
-          if (m == 0 && !ctx.wait(BAR_V_FULL + s, (pv_G / kStages) & 1)) return false;
-          if (!ctx.wait(BAR_P_FULL + m, pv_G & 1)) return false;
-          if (pv_first && pv_n >= 2 &&
-              !ctx.wait(BAR_O_EMPTY + 2 * m + (pv_n & 1), ((pv_n >> 1) - 1) & 1))
-            return false;
-          tc_fence_after_sync();
-          issue_pv(m, s, pv_n & 1, !pv_first);
-          if (m == 1) mma_commit(ctx.bar(BAR_KV_EMPTY + s));
-          if (pv_last) mma_commit(ctx.bar(BAR_O_FULL + 2 * m + (pv_n & 1)));
-          return true;
-        };
         int G = 0, n = 0;
         Item it;
         bool ok = true;
@@ -312,20 +356,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < it.n_tiles; ++j, ++G) {
             const int s = G % kStages;
             if (!(ok = ctx.wait(BAR_K_FULL + s, (G / kStages) & 1))) break;
-            tc_fence_after_sync();
-            if (pv_G >= 0 && !(ok = do_pv(0))) break;
-            issue_qk(0, qs, s);
-            mma_commit(ctx.bar(BAR_S_FULL + 0));
-            if (pv_G >= 0 && !(ok = do_pv(1))) break;
-            issue_qk(1, qs, s);
-            mma_commit(ctx.bar(BAR_S_FULL + 1));
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+              if (G > 0 && !(ok = ctx.wait(BAR_S_FREE + m, (G - 1) & 1))) break;
+              tc_fence_after_sync();
+              issue_qk(ctx, tmem, m, qs, s);
+              mma_commit(ctx.bar(BAR_S_FULL + m));
+            }
+            if (!ok) break;
+            if (pv_G >= 0 && !(ok = issue_pv_tile(ctx, tmem, pv_G, pv_n, pv_first, pv_last))) break;
             pv_G = G;
             pv_n = n;
             pv_first = j == 0;
             pv_last = j == it.n_tiles - 1;
           }
         }
-        if (ok && pv_G >= 0 && do_pv(0)) do_pv(1);
+        if (ok && pv_G >= 0) issue_pv_tile(ctx, tmem, pv_G, pv_n, pv_first, pv_last);
         // Every MMA issued must finish before the tensor memory is released.
         mma_commit(ctx.bar(BAR_MMA_DONE));
         volatile int never = 0;
@@ -339,20 +385,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = !skip;
       for (; ok && item_for(args, n, cta, &it); ++n) {
         const int qs = n & 1;
-        // positions first, so their latency overlaps the wait for the Q tile
-        int pq[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int tok = it.q0 + (i >> 1) * kTokensPerM + ((t + 64 * (i & 1)) >> 3);
-          pq[i] = tok < S ? load_position(args, it.b, tok) : -1;
-        }
         if (!(ok = ctx.wait_warp(BAR_Q_FULL + qs, (n >> 1) & 1))) break;
-#pragma unroll
+        const float2* tab = reinterpret_cast<const float2*>(smem + kOffTab + qs * kTabSlotBytes);
+#pragma unroll 1
         for (int i = 0; i < 4; ++i) {
           const int row = t + 64 * (i & 1);
-          if (pq[i] >= 0)
+          const int tl = (i >> 1) * kTokensPerM + (row >> 3);  // token within the item
+          if (it.q0 + tl < S)
             rope_row(smem + kOffQ + (2 * qs + (i >> 1)) * kTileBytes + row * 128, row,
-                     args.rope + static_cast<size_t>(pq[i]) * kRopePairs);
+                     tab + tl * kRopePairs);
         }
         fence_async_smem();
         __syncwarp();
@@ -367,6 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = wq * 32 + lane;  // row of the M tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + tmem_s(m);
+    const uint32_t tP = tmem + lane_off + tmem_p(m);
+    const uint32_t tO = tmem + lane_off + tmem_o(m);
     int G = 0, n = 0;
     Item it;
     bool ok = !skip;
@@ -374,7 +417,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tq = it.q0 + m * kTokensPerM + (r >> 3);
       const int tmin = it.q0 + m * kTokensPerM + wq * 4;  // tokens of this warp: tmin .. tmin+3
       const int tmax = tmin + 3;
-      const uint32_t tO = tmem + lane_off + tmem_o(m, n & 1);
       const float sink = __ldg(args.sinks + it.g * kGroup + (r & 7));
       const bool sink_off = isinf(sink) && sink < 0.f;
       float m_ref = sink_off ? -INFINITY : sink * kLog2e;
@@ -382,10 +424,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < it.n_tiles; ++j, ++G) {
         if (!(ok = ctx.wait_warp(BAR_S_FULL + m, G & 1))) break;
         tc_fence_after_sync();
-        const int kb = (it.jt0 + j) * kBlockN;
-        const bool wmask = (kb + kBlockN - 1 > tmin) || (W > 0 && kb <= tmax - W);
         uint32_t sv[128];
         tmem_ld128_split(tS, sv);
+        // S is in registers: let the next Q.K^T overwrite it.
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ctx.bar(BAR_S_FREE + m));
+        const int kb = (it.jt0 + j) * kBlockN;
+        const bool wmask = (kb + kBlockN - 1 > tmin) || (W > 0 && kb <= tmax - W);
         if (wmask) {
 #pragma unroll
           for (int i = 0; i < 128; ++i)
@@ -414,6 +460,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_ref = m_new;
           rescale = true;
         }
+        // The two softmax warpgroups take turns on the exponential unit (M
+        // tile 0 of tile G, M tile 1 of tile G, M tile 0 of tile G+1, ...):
+        // each one's loads, max and stores overlap the other's exponentials.
+        if (G > 0 || m == 1) {
+          if (!(ok = ctx.wait_warp(BAR_TURN + m, (m == 0 ? G - 1 : G) & 1))) break;
+        }
         // probabilities, packed to bf16 in place: sv[i] <- (p[2i], p[2i+1]);
         // scale-and-subtract and the row sum run on packed fp32 pairs
         const float mr = m_ref == -INFINITY ? 0.f : m_ref;
@@ -436,17 +488,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           sv[i] = pack_bf16x2(p0, p1);
           sv[i + 1] = pack_bf16x2(p2, p3);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ctx.bar(BAR_TURN + (m ^ 1)));
         {
           float a0, a1, a2, a3;
           f2_unpack(acc0, a0, a1);
           f2_unpack(acc1, a2, a3);
           l += (a0 + a1) + (a2 + a3);
         }
+        // P and O are free once the previous tile's P.V has completed.
+        if (G > 0 && !(ok = ctx.wait_warp(BAR_P_FREE + m, (G - 1) & 1))) break;
+        tc_fence_after_sync();
         {
           uint32_t pw[64];
 #pragma unroll
           for (int i = 0; i < 64; ++i) pw[i] = sv[i];
-          tmem_st64(tS, pw);
+          tmem_st64(tP, pw);
         }
         if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
@@ -482,38 +539,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     // below is always reached by all 128 threads; failed waits skip work.
     for (; item_for(args, n, cta, &it); ++n) {
       const int qs = n & 1;
-      const int ob = n & 1;
       bool ok = !skip && !*ctx.abort_flag;
 #pragma unroll 1
       for (int m = 0; m < 2; ++m) {
-        uint32_t ov[64];
-        const bool ok_o = ok && ctx.wait_warp(BAR_O_FULL + 2 * m + ob, (n >> 1) & 1);
+        const bool ok_o = ok && ctx.wait_warp(BAR_O_FULL + m, n & 1) &&
+                          ctx.wait_warp(BAR_L_FULL + m, n & 1);
         if (ok_o) {
-          tc_fence_after_sync();
-          tmem_ld64(tmem + lane_off + tmem_o(m, ob), ov);
-          tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(ctx.bar(BAR_O_EMPTY + 2 * m + ob));
-        }
-        const bool ok_l = ok_o && ctx.wait_warp(BAR_L_FULL + m, n & 1);
-        if (ok_l) {
-          const float l = l_smem[m * 128 + r];
+          const float inv_l = 1.f / l_smem[m * 128 + r];
           __syncwarp();
           if (lane == 0) mbar_arrive(ctx.bar(BAR_L_EMPTY + m));
-          const float inv_l = 1.f / l;
+          tc_fence_after_sync();
           uint8_t* stage = smem + kOffQ + (2 * qs + m) * kTileBytes;
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            uint32_t w[4];
+          for (int half = 0; half < 2; ++half) {
+            uint32_t ov[32];
+            tmem_ld32(tmem + lane_off + tmem_o(m) + 32 * half, ov);
+            if (half == 1) {
+              tc_fence_before_sync();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(ctx.bar(BAR_O_EMPTY + m));
+            }
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = pack_bf16x2(__uint_as_float(ov[8 * cc + 2 * e]) * inv_l,
-                                 __uint_as_float(ov[8 * cc + 2 * e + 1]) * inv_l);
-            *reinterpret_cast<uint4*>(stage + r * 128 + ((cc ^ (r & 7)) << 4)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                w[e] = pack_bf16x2(__uint_as_float(ov[8 * cc + 2 * e]) * inv_l,
+                                   __uint_as_float(ov[8 * cc + 2 * e + 1]) * inv_l);
+              const int chunk = 4 * half + cc;
+              *reinterpret_cast<uint4*>(stage + r * 128 + ((chunk ^ (r & 7)) << 4)) =
+                  make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
         }
-        ok = ok_l;
+        ok = ok_o;
       }
       fence_async_smem();
       named_barrier(1, 128);
@@ -558,10 +617,11 @@ namespace band {
 constexpr int kTokens = 16;
 constexpr int kSpan = 144;  // 128 keys before the tile + the tile's 16
 constexpr int kStages = 3;
-constexpr int kOutSlots = 4;  // output staging ring; a slot is reused 4 items later
+constexpr int kOutSlots = 3;  // output staging ring; a slot is reused 3 items later
 constexpr uint32_t kQBytes = 128 * 128;
 constexpr uint32_t kKVBytes = kSpan * 128;
-constexpr uint32_t kStageBytes = kQBytes + 2 * kKVBytes;
+constexpr uint32_t kTabBytes = kTokens * kRopePairs * 8;  // table rows of the 16 tokens
+constexpr uint32_t kStageBytes = kQBytes + 2 * kKVBytes + kTabBytes;
 constexpr uint32_t kOffStage = 0;
 constexpr uint32_t kOffOut = kStages * kStageBytes;          // [kOutSlots] staging tiles
 constexpr uint32_t kOffL = kOffOut + kOutSlots * kQBytes;    // float [2][128]
@@ -600,6 +660,7 @@ struct Ctx {
   __device__ uint32_t q(int s) const { return sbase + kOffStage + s * kStageBytes; }
   __device__ uint32_t k(int s) const { return q(s) + kQBytes; }
   __device__ uint32_t v(int s) const { return q(s) + kQBytes + kKVBytes; }
+  __device__ uint32_t tab(int s) const { return q(s) + kQBytes + 2 * kKVBytes; }
 };
 
 struct Item {
@@ -616,6 +677,24 @@ __device__ __forceinline__ bool item_for(const PrefillArgs& a, int k, int cta, I
   const int rem = idx % per_tile;
   it->g = rem % kNumKvHeads;
   it->b = rem / kNumKvHeads;
+  return true;
+}
+
+// O (+)= P V for item p (9 MMAs of K = 16 over the 144-key span), then the
+// commits that publish O and release the item's stage.
+__device__ __forceinline__ bool issue_pv(const Ctx& ctx, uint32_t tmem, int p) {
+  constexpr uint32_t idesc_pv = idesc_bf16(128, kHeadDim, true);
+  const int m = p & 1, s = p % kStages;
+  if (!ctx.wait(BAR_V_FULL + s, (p / kStages) & 1)) return false;
+  if (!ctx.wait(BAR_P_FULL + m, (p >> 1) & 1)) return false;
+  if (p >= 2 && !ctx.wait(BAR_O_EMPTY + m, ((p >> 1) - 1) & 1)) return false;
+  tc_fence_after_sync();
+#pragma unroll
+  for (int kk = 0; kk < kSpan / 16; ++kk)
+    mma_bf16_ts(tmem + tmem_o(m), tmem + tmem_s(m) + 8 * kk, sdesc_sw128(ctx.v(s) + 2048 * kk),
+                idesc_pv, kk > 0 ? 1u : 0u);
+  mma_commit(ctx.bar(BAR_O_FULL + m));
+  mma_commit(ctx.bar(BAR_EMPTY + s));
   return true;
 }
 
@@ -686,10 +765,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               !ctx.wait(band::BAR_EMPTY + s, ((k / band::kStages) - 1) & 1))
             break;
           const int kb = it.q0 - 128;
-          mbar_arrive_expect_tx(ctx.bar(band::BAR_QK_FULL + s), band::kQBytes + band::kKVBytes);
+          const uint32_t tab_bytes =
+              kRopePairs * 8 * static_cast<uint32_t>(min(band::kTokens, S - it.q0));
+          mbar_arrive_expect_tx(ctx.bar(band::BAR_QK_FULL + s),
+                                band::kQBytes + band::kKVBytes + tab_bytes);
           tma_load_4d(ctx.q(s), &maps.q, ctx.bar(band::BAR_QK_FULL + s), 0, it.g * kGroup, it.q0,
                       it.b);
           tma_load_4d(ctx.k(s), &maps.k_band, ctx.bar(band::BAR_QK_FULL + s), 0, it.g, kb, it.b);
+          stage_rope_rows<band::kTokens>(args, it.b, it.q0, ctx.tab(s),
+                                         ctx.bar(band::BAR_QK_FULL + s));
           mbar_arrive_expect_tx(ctx.bar(band::BAR_V_FULL + s), band::kKVBytes);
           tma_load_4d(ctx.v(s), &maps.v_band, ctx.bar(band::BAR_V_FULL + s), 0, it.g, kb, it.b);
         }
@@ -707,21 +791,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // -------------------------------------------------------------- MMA issuer
       if (lane == 0 && !skip) {
         constexpr uint32_t idesc_qk = idesc_bf16(128, band::kSpan, false);
-        constexpr uint32_t idesc_pv = idesc_bf16(128, kHeadDim, true);
-        auto do_pv = [&](int p) -> bool {
-          const int m = p & 1, s = p % band::kStages;
-          if (!ctx.wait(band::BAR_V_FULL + s, (p / band::kStages) & 1)) return false;
-          if (!ctx.wait(band::BAR_P_FULL + m, (p >> 1) & 1)) return false;
-          if (p >= 2 && !ctx.wait(band::BAR_O_EMPTY + m, ((p >> 1) - 1) & 1)) return false;
-          tc_fence_after_sync();
-#pragma unroll
-          for (int kk = 0; kk < band::kSpan / 16; ++kk)
-            mma_bf16_ts(tmem + band::tmem_o(m), tmem + band::tmem_s(m) + 8 * kk,
-                        sdesc_sw128(ctx.v(s) + 2048 * kk), idesc_pv, kk > 0 ? 1u : 0u);
-          mma_commit(ctx.bar(band::BAR_O_FULL + m));
-          mma_commit(ctx.bar(band::BAR_EMPTY + s));
-          return true;
-        };
         int k = 0;
         band::Item it;
         bool ok = true;
@@ -736,9 +805,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_bf16_ss(tmem + band::tmem_s(m), sdesc_sw128(ctx.q(s) + 32 * kk),
                         sdesc_sw128(ctx.k(s) + 32 * kk), idesc_qk, kk > 0 ? 1u : 0u);
           mma_commit(ctx.bar(band::BAR_S_FULL + m));
-          if (k > 0 && !(ok = do_pv(k - 1))) break;
+          if (k > 0 && !(ok = band::issue_pv(ctx, tmem, k - 1))) break;
         }
-        if (ok && k > 0) do_pv(k - 1);
+        if (ok && k > 0) band::issue_pv(ctx, tmem, k - 1);
         mma_commit(ctx.bar(band::BAR_MMA_DONE));
         volatile int never = 0;
         mbar_wait(ctx.bar(band::BAR_MMA_DONE), 0, &never, nullptr, 0, kWaitTimeoutNs);
@@ -750,19 +819,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = !skip;
       for (int k = 0; ok && band::item_for(args, k, cta, &it); ++k) {
         const int s = k % band::kStages;
-        int pq[2];
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const int tok = it.q0 + ((t + 64 * rr) >> 3);
-          pq[rr] = tok < S ? load_position(args, it.b, tok) : -1;
-        }
         if (!(ok = ctx.wait_warp(band::BAR_QK_FULL + s, (k / band::kStages) & 1))) break;
         uint8_t* qt = smem + band::kOffStage + s * band::kStageBytes;
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr)
-          if (pq[rr] >= 0)
-            rope_row(qt + (t + 64 * rr) * 128, t + 64 * rr,
-                     args.rope + static_cast<size_t>(pq[rr]) * kRopePairs);
+        const float2* tab =
+            reinterpret_cast<const float2*>(qt + band::kQBytes + 2 * band::kKVBytes);
+#pragma unroll 1
+        for (int rr = 0; rr < 2; ++rr) {
+          const int row = t + 64 * rr;
+          if (it.q0 + (row >> 3) < S) rope_row(qt + row * 128, row, tab + (row >> 3) * kRopePairs);
+        }
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(ctx.bar(band::BAR_READY + s));
@@ -790,23 +855,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after_sync();
       uint32_t sv[band::kSpan];
       tmem_ld144_split(tS, sv);
-      float mx = sink_off ? -INFINITY : sink * kLog2e;
+      // Columns that can be masked: those before c_lo and after c_hi. With
+      // W = 128 and q0 >= 128 that is only [0, 17) and [128, 144).
+      // (Only the executed branch occupies the instruction cache, so the
+      // common case stays short.)
+      if (W == 128 && it.q0 >= 128) {
 #pragma unroll
-      for (int c = 0; c < band::kSpan; ++c) {
-        const float x = (c >= c_lo && c <= c_hi) ? __uint_as_float(sv[c]) * kScaleLog2 : -INFINITY;
-        sv[c] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+        for (int c = 0; c < 17; ++c)
+          if (c < c_lo) sv[c] = __float_as_uint(-INFINITY);
+#pragma unroll
+        for (int c = 128; c < band::kSpan; ++c)
+          if (c > c_hi) sv[c] = __float_as_uint(-INFINITY);
+      } else {
+#pragma unroll
+        for (int c = 0; c < band::kSpan; ++c)
+          if (c < c_lo || c > c_hi) sv[c] = __float_as_uint(-INFINITY);
       }
+      float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < band::kSpan; c += 8) {
+        m0 = fmax3(m0, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
+        m1 = fmax3(m1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
+        m2 = fmax3(m2, __uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
+        m3 = fmax3(m3, __uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
+      }
+      const float mx = fmaxf(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * kScaleLog2,
+                             sink_off ? -INFINITY : sink * kLog2e);
       const float mr = mx == -INFINITY ? 0.f : mx;
-      float l0 = sink_off ? 0.f : ex2_approx(sink * kLog2e - mr), l1 = 0.f;
+      const uint64_t c2 = f2_pack(kScaleLog2, kScaleLog2);
+      const uint64_t nm2 = f2_pack(-mr, -mr);
+      uint64_t acc0 = f2_pack(sink_off ? 0.f : ex2_approx(sink * kLog2e - mr), 0.f);
+      uint64_t acc1 = f2_pack(0.f, 0.f);
       // probabilities packed to bf16 in place: sv[c] <- (p[2c], p[2c+1])
 #pragma unroll
-      for (int c = 0; c < band::kSpan / 2; ++c) {
-        const float p0 = ex2_approx(__uint_as_float(sv[2 * c]) - mr);
-        const float p1 = ex2_approx(__uint_as_float(sv[2 * c + 1]) - mr);
-        l0 += p0;
-        l1 += p1;
+      for (int c = 0; c < band::kSpan / 2; c += 2) {
+        float x0, x1, x2, x3;
+        f2_unpack(ffma2(f2_pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), c2,
+                        nm2),
+                  x0, x1);
+        f2_unpack(ffma2(f2_pack(__uint_as_float(sv[2 * c + 2]), __uint_as_float(sv[2 * c + 3])),
+                        c2, nm2),
+                  x2, x3);
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+        acc0 = fadd2(acc0, f2_pack(p0, p1));
+        acc1 = fadd2(acc1, f2_pack(p2, p3));
         sv[c] = pack_bf16x2(p0, p1);
+        sv[c + 1] = pack_bf16x2(p2, p3);
+      }
+      float l0, l1;
+      {
+        float a0, a1, a2, a3;
+        f2_unpack(acc0, a0, a1);
+        f2_unpack(acc1, a2, a3);
+        l0 = a0 + a2;
+        l1 = a1 + a3;
       }
       {
         uint32_t a[64], b8[8];
@@ -836,30 +939,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; band::item_for(args, k, cta, &it); ++k) {
       const int m = k & 1, i = k >> 1;
       uint8_t* stage = smem + band::kOffOut + (k % band::kOutSlots) * band::kQBytes;
-      bool ok = !skip && !*ctx.abort_flag && ctx.wait_warp(band::BAR_O_FULL + m, i & 1);
-      uint32_t ov[64];
+      bool ok = !skip && !*ctx.abort_flag && ctx.wait_warp(band::BAR_O_FULL + m, i & 1) &&
+                ctx.wait_warp(band::BAR_L_FULL + m, i & 1);
       if (ok) {
-        tc_fence_after_sync();
-        tmem_ld64(tmem + lane_off + band::tmem_o(m), ov);
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(ctx.bar(band::BAR_O_EMPTY + m));
-      }
-      ok = ok && ctx.wait_warp(band::BAR_L_FULL + m, i & 1);
-      if (ok) {
-        const float l = l_smem[m * 128 + r];
+        const float inv_l = 1.f / l_smem[m * 128 + r];
         __syncwarp();
         if (lane == 0) mbar_arrive(ctx.bar(band::BAR_L_EMPTY + m));
-        const float inv_l = 1.f / l;
+        tc_fence_after_sync();
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          uint32_t w[4];
+        for (int half = 0; half < 2; ++half) {
+          uint32_t ov[32];
+          tmem_ld32(tmem + lane_off + band::tmem_o(m) + 32 * half, ov);
+          if (half == 1) {
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ctx.bar(band::BAR_O_EMPTY + m));
+          }
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(ov[8 * cc + 2 * e]) * inv_l,
-                               __uint_as_float(ov[8 * cc + 2 * e + 1]) * inv_l);
-          *reinterpret_cast<uint4*>(stage + r * 128 + ((cc ^ (r & 7)) << 4)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack_bf16x2(__uint_as_float(ov[8 * cc + 2 * e]) * inv_l,
+                                 __uint_as_float(ov[8 * cc + 2 * e + 1]) * inv_l);
+            const int chunk = 4 * half + cc;
+            *reinterpret_cast<uint4*>(stage + r * 128 + ((chunk ^ (r & 7)) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
       fence_async_smem();
