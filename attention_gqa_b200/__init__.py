@@ -20,7 +20,8 @@ import os
 
 import torch
 
-__all__ = ["prefill", "decode", "prefill_workspace_bytes", "decode_workspace_bytes", "check", "init", "rope_table",
+__all__ = ["prefill", "decode", "decode_noalloc", "prefill_workspace_bytes",
+           "decode_workspace_bytes", "check", "init", "rope_table",
            "library_path", "GptossAttnError", "NUM_HEADS", "NUM_KV_HEADS", "HEAD_DIM",
            "MAX_POSITION"]
 
@@ -241,6 +242,33 @@ def decode(q, kcache, vcache, sinks, lengths, window: int = 0, out=None, workspa
                                 _stream_handle(stream))
     _raise(st, "gptoss_attn_decode")
     return dev_out
+
+
+def decode_noalloc(q, kcache, vcache, sinks, lengths, window: int = 0, out=None,
+                   stream=None) -> torch.Tensor:
+    """decode() for callers that cannot allocate device memory: the split
+    partials live in the library's fixed device array (GPTOSS_ATTN_NOALLOC_
+    SCRATCH_BYTES) instead of a workspace. Device tensors only; pass `out` to
+    allocate nothing here either. Calls whose kernels overlap in time race."""
+    lib = _load()
+    fn = lib.gptoss_attn_decode_noalloc
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, vp]
+    fn.restype = i32
+    device = q.device
+    if device.type != "cuda":
+        raise ValueError("decode_noalloc takes device tensors")
+    for name, t, dt in (("q", q, torch.bfloat16), ("kcache", kcache, torch.bfloat16),
+                        ("vcache", vcache, torch.bfloat16), ("sinks", sinks, torch.float32),
+                        ("lengths", lengths, torch.int32)):
+        _dev(t, dt, name, device)
+    B, L = q.shape[0], kcache.shape[1]
+    if out is None:
+        out = torch.empty((B, NUM_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=device)
+    st = fn(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), sinks.data_ptr(),
+            lengths.data_ptr(), int(window), out.data_ptr(), B, L, _stream_handle(stream))
+    _raise(st, "gptoss_attn_decode_noalloc")
+    return out
 
 
 def check(stream=None) -> None:

@@ -151,6 +151,37 @@ int gptoss_attn_decode(const void* q, const void* kcache, const void* vcache, co
                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Allocation-free decode. The gpt-oss pages have no counterpart: this entry
+ * point exists for callers that cannot allocate device memory while they
+ * decode, such as code recording a CUDA graph (allocation is not allowed
+ * during stream capture), serving engines that give all device memory to
+ * their own pool up front, and latency-bound loops that cannot pay for an
+ * allocation's synchronization.
+ *
+ * Same operation and arguments as gptoss_attn_decode() without the
+ * workspace: the split partials live in a fixed array of
+ * GPTOSS_ATTN_NOALLOC_SCRATCH_BYTES bytes that is part of the library's
+ * device image, held on every GPU that loads the library until the process
+ * exits. Sizes whose partials do not fit (batch * 64 heads * splits * 264
+ * bytes, see gptoss_attn_decode_workspace_bytes()) are rejected with
+ * GPTOSS_ATTN_ERR_SMALL_WORKSPACE before any work is enqueued. The call
+ * allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.
+ * Every call shares the array, and a call clears only its error word before
+ * launching, so calls whose kernels overlap in time on the GPU race: issue
+ * them on one stream or otherwise serialize them. Device-side conditions of
+ * this path (a length outside [0, max_len], which is clamped; a pipeline
+ * timeout) are not reported by gptoss_attn_check().
+ */
+#define GPTOSS_ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+int gptoss_attn_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                               const float* sinks, const int32_t* len, int window, void* out,
+                               int batch, int max_len, cudaStream_t stream);
+
+/*
  * Synchronizes `stream`, then reads and clears the current device's error
  * word. Returns GPTOSS_ATTN_OK, GPTOSS_ATTN_ERR_DEVICE_TIMEOUT,
  * GPTOSS_ATTN_ERR_BAD_POSITION, GPTOSS_ATTN_ERR_BAD_LENGTH or
