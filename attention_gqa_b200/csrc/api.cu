@@ -158,8 +158,8 @@ int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float
   args.n_qtiles = (seqlen + 31) / 32;
   args.n_items = prefill_items(batch, seqlen, args.window);
   args.grid = g_state[dev].num_sms;
-  if (launch_rope_keys(k, pos, args.rope, workspace, static_cast<int64_t>(batch) * seqlen,
-                       args.grid * 8, args.err, stream) != cudaSuccess)
+  if (launch_rope_rows(k, pos, args.rope, workspace, static_cast<int64_t>(batch) * seqlen,
+                       kNumKvHeads, args.grid * 8, args.err, stream) != cudaSuccess)
     return GPTOSS_ATTN_ERR_LAUNCH;
   return launch_prefill(maps, args, stream) == cudaSuccess ? GPTOSS_ATTN_OK
                                                            : GPTOSS_ATTN_ERR_LAUNCH;

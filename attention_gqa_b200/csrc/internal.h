@@ -53,9 +53,11 @@ cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cud
 // Fills the rotary table [kMaxPosition][32] of (cos, sin).
 cudaError_t launch_rope_table(float2* table, cudaStream_t stream);
 
-// Rotates the key rows of k [n_tokens][8][64] (bf16) by pos[token] into k_rot.
-cudaError_t launch_rope_keys(const void* k, const int32_t* pos, const float2* table, void* k_rot,
-                             int64_t n_tokens, int grid_cap, int* err, cudaStream_t stream);
+// Rotates the rows of x [n_tokens][heads][64] (bf16; heads = 8 for keys or 64
+// for queries) by pos[token] into x_rot.
+cudaError_t launch_rope_rows(const void* x, const int32_t* pos, const float2* table, void* x_rot,
+                             int64_t n_tokens, int heads, int grid_cap, int* err,
+                             cudaStream_t stream);
 
 struct DecodeArgs {
   const uint16_t* q;       // [B][64][64] bf16, un-rotated

@@ -12,17 +12,24 @@
 // which balances the causal triangle without a global counter.
 //
 // Roles (512 threads, four warpgroups):
-//   WG0 warp 0    TMA producer: Q per item into a 2-slot buffer, K/V tiles of
-//                 128 keys through a kStages-deep ring.
-//   WG0 warp 1    TMEM owner and tcgen05 issuer (one thread): S = Q K^T
-//                 (SS, K-major) and O += P V (A = P from TMEM, B = V MN-major).
-//   WG0 warps 2-3 RoPE: rotate the Q rows of each item in shared memory, from
-//                 an fp64-built (cos, sin) table. Keys arrive already rotated
-//                 (a pre-pass rotates each key once per layer).
+//   WG0 warp 0    TMA producer of Q per item (2-slot buffer, with the
+//                 rotary-table rows of its tokens) and of K tiles of 128 keys
+//                 through a kStages-deep ring; warp 3 produces the V tiles.
+//                 A K stage is released after both M tiles' Q.K^T, a V stage
+//                 after both P.V, so K runs further ahead than V.
+//   WG0 warps 1-2 one tcgen05 issuer thread per M tile m (warp 1 also owns
+//                 the tensor memory): S_m = Q_m K^T (SS, K-major) and
+//                 O_m += P_m V (A = P from TMEM, B = V MN-major). Separate
+//                 issuers keep each M tile's pipeline independent of the
+//                 other's progress; the tensor core interleaves the streams.
 //   WG1, WG2      softmax for M tile 0 / 1 (thread = TMEM lane = one query row):
 //                 one 128-column TMEM load per tile, sink-seeded online softmax
-//                 in log2 units, bf16 P written back over S.
-//   WG3           epilogue: O / l -> bf16 -> swizzled staging -> TMA store.
+//                 in log2 units, bf16 P to TMEM; after an item's last tile the
+//                 same warpgroup normalises O and stores it (bf16, TMA) through
+//                 its half of the item's Q slot.
+//   WG3           RoPE: rotates the Q rows of each item in shared memory from
+//                 an fp64-built (cos, sin) table. Keys arrive already rotated
+//                 (a pre-pass rotates each key once per layer).
 // TMEM (512 columns): S0 [0,128), S1 [128,256), P0 [256,320), P1 [320,384),
 // O0 [384,448), O1 [448,512). The softmax releases S right after loading it,
 // so Q K^T of tile j+1 overlaps the softmax of tile j and P.V of tile j
@@ -40,7 +47,7 @@ namespace {
 constexpr int kBlockQ = 32;      // query tokens per work item
 constexpr int kTokensPerM = 16;  // tokens per M=128 tile (x 8 heads)
 constexpr int kBlockN = 128;     // keys per K/V tile
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kThreads = 512;
 constexpr uint32_t kTileBytes = 128 * 128;  // 128 rows of 64 bf16
 
@@ -61,36 +68,43 @@ static_assert(2 * 128 * kRegsLight + 2 * 128 * kRegsSoftmax <= 512 * 128, "regis
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kScaleLog2 = 0.125f * kLog2e;  // 1/sqrt(64) * log2(e)
 constexpr float kRescaleThreshold = 8.0f;      // log2 units
+// Exp-loop step (of 64 column pairs) at which a softmax warpgroup releases the
+// exponential unit to the other one (measured best at about 5/8 of the loop).
+constexpr int kTurnHandOff = 38;
+
+// Rotary-table rows in shared memory: 32 (cos, sin) pairs plus 16 bytes of
+// padding, so the rows of the four tokens a warp touches sit in different banks.
+constexpr uint32_t kTabRowBytes = kRopePairs * 8 + 16;
+constexpr int kTabRowPairs = static_cast<int>(kTabRowBytes / 8);
 
 enum : int {
   BAR_Q_FULL = 0,                        // [2] slot loaded
   BAR_Q_READY = BAR_Q_FULL + 2,          // [2] slot rotated
-  BAR_Q_EMPTY = BAR_Q_READY + 2,         // [2] slot's output stored
+  BAR_Q_EMPTY = BAR_Q_READY + 2,         // [2] slot's outputs stored (both halves)
   BAR_K_FULL = BAR_Q_EMPTY + 2,          // [kStages]
   BAR_V_FULL = BAR_K_FULL + kStages,     // [kStages]
-  BAR_KV_EMPTY = BAR_V_FULL + kStages,   // [kStages]
-  BAR_S_FULL = BAR_KV_EMPTY + kStages,   // [2] per M tile: S written
+  BAR_K_EMPTY = BAR_V_FULL + kStages,    // [kStages] both M tiles' Q.K^T done with the stage
+  BAR_V_EMPTY = BAR_K_EMPTY + kStages,   // [kStages] both M tiles' P.V done with the stage
+  BAR_S_FULL = BAR_V_EMPTY + kStages,    // [2] per M tile: S written
   BAR_S_FREE = BAR_S_FULL + 2,           // [2] S read by the softmax
   BAR_P_FULL = BAR_S_FREE + 2,           // [2] P written
-  BAR_P_FREE = BAR_P_FULL + 2,           // [2] P.V done (P and O free)
+  BAR_P_FREE = BAR_P_FULL + 2,           // [2] P.V done (P free)
   BAR_O_FULL = BAR_P_FREE + 2,           // [2] item's O complete
-  BAR_O_EMPTY = BAR_O_FULL + 2,          // [2] item's O read by the epilogue
-  BAR_L_FULL = BAR_O_EMPTY + 2,          // [2]
-  BAR_L_EMPTY = BAR_L_FULL + 2,          // [2]
-  BAR_TURN = BAR_L_EMPTY + 2,            // [2] exp-loop turn of softmax warpgroup m
-  BAR_MMA_DONE = BAR_TURN + 2,
-  NUM_BARS
+  BAR_STAGED = BAR_O_FULL + 2,           // [2] item's normalised O in shared memory
+  BAR_TURN = BAR_STAGED + 2,             // [2] exp-loop turn of softmax warpgroup m
+  BAR_MMA_DONE = BAR_TURN + 2,           // [2] per issuer
+  NUM_BARS = BAR_MMA_DONE + 2
 };
 
 constexpr uint32_t kOffQ = 0;  // [2 slots][2 halves] tiles
 constexpr uint32_t kOffK = kOffQ + 4 * kTileBytes;
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
-constexpr uint32_t kOffL = kOffV + kStages * kTileBytes;  // float [2][128]
-constexpr uint32_t kOffTab = kOffL + 2 * 128 * 4;  // float2 [2 slots][32 tokens][32]
-constexpr uint32_t kTabSlotBytes = kBlockQ * kRopePairs * 8;
+constexpr uint32_t kOffTab = kOffV + kStages * kTileBytes;  // [2 slots][32 tokens] table rows
+constexpr uint32_t kTabSlotBytes = kBlockQ * kTabRowBytes;
 constexpr uint32_t kOffBar = kOffTab + 2 * kTabSlotBytes;
 constexpr uint32_t kOffMisc = kOffBar + NUM_BARS * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 struct Ctx {
   uint32_t sbase;
@@ -135,37 +149,46 @@ __device__ __forceinline__ bool item_for(const PrefillArgs& a, int k, int cta, I
 // row index r) by the (cos, sin) table row `cs` of its position, in place.
 // Both live in shared memory: the producer stages the table rows an item
 // needs (one per token) next to its Q tile.
+// Rotates, in place, the 16-byte chunks c and c+4 (elements 8c..8c+7 and
+// their partners 8c+32..8c+39) of a 64-element row stored at `row` (128 bytes,
+// 128B-swizzled with row index r), with the (cos, sin) of pairs 8c..8c+7.
+__device__ __forceinline__ void rope_chunk(uint8_t* row, int r, int c, const float (&cv)[8],
+                                           const float (&sv)[8]) {
+  uint4* plo = reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4));
+  uint4* phi = reinterpret_cast<uint4*>(row + (((c + 4) ^ (r & 7)) << 4));
+  const uint4 a = *plo, h = *phi;
+  const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+  const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+  uint32_t ya[4], yh[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float x1l = bf16lo_to_f32(aw[e]), x1h = bf16hi_to_f32(aw[e]);
+    const float x2l = bf16lo_to_f32(hw[e]), x2h = bf16hi_to_f32(hw[e]);
+    const float cl = cv[2 * e], ch = cv[2 * e + 1], sl = sv[2 * e], sh = sv[2 * e + 1];
+    ya[e] = pack_bf16x2(fmaf(x1l, cl, -x2l * sl), fmaf(x1h, ch, -x2h * sh));
+    yh[e] = pack_bf16x2(fmaf(x2l, cl, x1l * sl), fmaf(x2h, ch, x1h * sh));
+  }
+  *plo = make_uint4(ya[0], ya[1], ya[2], ya[3]);
+  *phi = make_uint4(yh[0], yh[1], yh[2], yh[3]);
+}
+
+// Rotates a whole row with the table row `cs` of its position (both in shared memory).
 __device__ __forceinline__ void rope_row(uint8_t* row, int r, const float2* cs) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    uint4* plo = reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4));
-    uint4* phi = reinterpret_cast<uint4*>(row + (((c + 4) ^ (r & 7)) << 4));
     const float4* t4 = reinterpret_cast<const float4*>(cs + 8 * c);
     const float4 t0 = t4[0], t1 = t4[1], t2 = t4[2], t3 = t4[3];
-    const uint4 a = *plo, h = *phi;
     const float cv[8] = {t0.x, t0.z, t1.x, t1.z, t2.x, t2.z, t3.x, t3.z};
     const float sv[8] = {t0.y, t0.w, t1.y, t1.w, t2.y, t2.w, t3.y, t3.w};
-    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-    const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
-    uint32_t ya[4], yh[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float x1l = bf16lo_to_f32(aw[e]), x1h = bf16hi_to_f32(aw[e]);
-      const float x2l = bf16lo_to_f32(hw[e]), x2h = bf16hi_to_f32(hw[e]);
-      const float cl = cv[2 * e], ch = cv[2 * e + 1], sl = sv[2 * e], sh = sv[2 * e + 1];
-      ya[e] = pack_bf16x2(fmaf(x1l, cl, -x2l * sl), fmaf(x1h, ch, -x2h * sh));
-      yh[e] = pack_bf16x2(fmaf(x2l, cl, x1l * sl), fmaf(x2h, ch, x1h * sh));
-    }
-    *plo = make_uint4(ya[0], ya[1], ya[2], ya[3]);
-    *phi = make_uint4(yh[0], yh[1], yh[2], yh[3]);
+    rope_chunk(row, r, c, cv, sv);
   }
 }
 
 // Stages the rotary-table rows of tokens q0 .. q0+n-1 of sequence b (one
-// 256-byte row each; the 8 heads of a token share its position) into
-// shared memory at `dst`, completing on `bar`. Returns the bytes requested;
-// tokens past the sequence end are skipped. Run by one thread.
-template <int kTokensPerItem>
+// 256-byte row each, kRowStride bytes apart in shared memory; the 8 heads of
+// a token share its position) at `dst`, completing on `bar`. Returns the
+// bytes requested; tokens past the sequence end are skipped. Run by one thread.
+template <int kTokensPerItem, uint32_t kRowStride>
 __device__ __forceinline__ uint32_t stage_rope_rows(const PrefillArgs& a, int b, int q0,
                                                     uint32_t dst, uint32_t bar) {
   constexpr uint32_t kRowBytes = kRopePairs * sizeof(float2);
@@ -186,7 +209,7 @@ __device__ __forceinline__ uint32_t stage_rope_rows(const PrefillArgs& a, int b,
         atomicOr(a.err, kErrPosition);
         pt = pt < 0 ? 0 : kMaxPosition - 1;
       }
-      bulk_load(dst + (t0 + t) * kRowBytes, a.rope + static_cast<size_t>(pt) * kRopePairs,
+      bulk_load(dst + (t0 + t) * kRowStride, a.rope + static_cast<size_t>(pt) * kRopePairs,
                 kRowBytes, bar);
       bytes += kRowBytes;
     }
@@ -209,27 +232,25 @@ __device__ __forceinline__ void issue_qk(const Ctx& ctx, uint32_t tmem, int m, i
                 kk > 0 ? 1u : 0u);
 }
 
-// O_m (+)= P_m V for both M tiles of global tile G (item n), then the commits
-// that release P, the K/V stage and, after an item's last tile, O.
-__device__ __forceinline__ bool issue_pv_tile(const Ctx& ctx, uint32_t tmem, int G, int n,
-                                              bool first, bool last) {
+// O_m (+)= P_m V for global tile G, then the commits that release P, this
+// M tile's use of the K/V stage and, after an item's last tile, O. The first
+// tile of an item overwrites O: the softmax publishes that tile's P only after
+// it has read out the previous item's O.
+__device__ __forceinline__ bool issue_pv(const Ctx& ctx, uint32_t tmem, int m, int G, bool first,
+                                         bool last) {
   constexpr uint32_t idesc = idesc_bf16(128, kHeadDim, true);
   const int s = G % kStages;
   if (!ctx.wait(BAR_V_FULL + s, (G / kStages) & 1)) return false;
+  if (!ctx.wait(BAR_P_FULL + m, G & 1)) return false;
+  tc_fence_after_sync();
   const uint32_t va = ctx.sbase + kOffV + s * kTileBytes;
 #pragma unroll
-  for (int m = 0; m < 2; ++m) {
-    if (!ctx.wait(BAR_P_FULL + m, G & 1)) return false;
-    if (first && n >= 1 && !ctx.wait(BAR_O_EMPTY + m, (n - 1) & 1)) return false;
-    tc_fence_after_sync();
-#pragma unroll
-    for (int kk = 0; kk < kBlockN / 16; ++kk)
-      mma_bf16_ts(tmem + tmem_o(m), tmem + tmem_p(m) + 8 * kk, sdesc_sw128(va + 2048 * kk), idesc,
-                  (!first || kk > 0) ? 1u : 0u);
-    mma_commit(ctx.bar(BAR_P_FREE + m));
-    if (last) mma_commit(ctx.bar(BAR_O_FULL + m));
-  }
-  mma_commit(ctx.bar(BAR_KV_EMPTY + s));
+  for (int kk = 0; kk < kBlockN / 16; ++kk)
+    mma_bf16_ts(tmem + tmem_o(m), tmem + tmem_p(m) + 8 * kk, sdesc_sw128(va + 2048 * kk), idesc,
+                (!first || kk > 0) ? 1u : 0u);
+  mma_commit(ctx.bar(BAR_P_FREE + m));
+  if (last) mma_commit(ctx.bar(BAR_O_FULL + m));
+  mma_commit(ctx.bar(BAR_V_EMPTY + s));
   return true;
 }
 
@@ -243,7 +264,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   ctx.abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   ctx.err = args.err;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-  float* l_smem = reinterpret_cast<float*>(smem + kOffL);
 
   const int warp = static_cast<int>(threadIdx.x >> 5);
   const int lane = static_cast<int>(threadIdx.x & 31);
@@ -254,24 +274,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(ctx.bar(BAR_Q_FULL + i), 1);
-      mbar_init(ctx.bar(BAR_Q_READY + i), 2);
-      mbar_init(ctx.bar(BAR_Q_EMPTY + i), 1);
+      mbar_init(ctx.bar(BAR_Q_READY + i), 4);
+      mbar_init(ctx.bar(BAR_Q_EMPTY + i), 2);
       mbar_init(ctx.bar(BAR_S_FULL + i), 1);
       mbar_init(ctx.bar(BAR_S_FREE + i), 4);
       mbar_init(ctx.bar(BAR_P_FULL + i), 4);
       mbar_init(ctx.bar(BAR_P_FREE + i), 1);
       mbar_init(ctx.bar(BAR_O_FULL + i), 1);
-      mbar_init(ctx.bar(BAR_O_EMPTY + i), 4);
-      mbar_init(ctx.bar(BAR_L_FULL + i), 4);
-      mbar_init(ctx.bar(BAR_L_EMPTY + i), 4);
+      mbar_init(ctx.bar(BAR_STAGED + i), 4);
       mbar_init(ctx.bar(BAR_TURN + i), 4);
+      mbar_init(ctx.bar(BAR_MMA_DONE + i), 1);
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(ctx.bar(BAR_K_FULL + s), 1);
       mbar_init(ctx.bar(BAR_V_FULL + s), 1);
-      mbar_init(ctx.bar(BAR_KV_EMPTY + s), 1);
+      mbar_init(ctx.bar(BAR_K_EMPTY + s), 2);
+      mbar_init(ctx.bar(BAR_V_EMPTY + s), 2);
     }
-    mbar_init(ctx.bar(BAR_MMA_DONE), 1);
     // A pipeline timeout earlier left the error word set: skip the work.
     *ctx.abort_flag = (*reinterpret_cast<volatile int*>(args.err) & kErrTimeout) ? 1 : 0;
     fence_barrier_init();
@@ -294,7 +313,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && !skip) {
         prefetch_tensormap(&maps.q);
         prefetch_tensormap(&maps.k);
-        prefetch_tensormap(&maps.v);
         int G = 0, n = 0, nq = 0;
         Item it;
         bool ok = true;
@@ -307,43 +325,63 @@ __global__ void __launch_bounds__(kThreads, 1)
                       it.q0, it.b);
           tma_load_4d(ctx.q_tile(qs, 1), &maps.q, ctx.bar(BAR_Q_FULL + qs), 0, it.g * kGroup,
                       it.q0 + kTokensPerM, it.b);
-          stage_rope_rows<kBlockQ>(args, it.b, it.q0, ctx.sbase + kOffTab + qs * kTabSlotBytes,
-                                   ctx.bar(BAR_Q_FULL + qs));
+          stage_rope_rows<kBlockQ, kTabRowBytes>(args, it.b, it.q0,
+                                                 ctx.sbase + kOffTab + qs * kTabSlotBytes,
+                                                 ctx.bar(BAR_Q_FULL + qs));
           nq = n + 1;
           for (int j = 0; j < it.n_tiles; ++j) {
             const int s = G % kStages;
-            if (G >= kStages && !(ok = ctx.wait(BAR_KV_EMPTY + s, ((G / kStages) - 1) & 1)))
+            if (G >= kStages && !(ok = ctx.wait(BAR_K_EMPTY + s, ((G / kStages) - 1) & 1)))
               break;
-            const int kb = (it.jt0 + j) * kBlockN;
             mbar_arrive_expect_tx(ctx.bar(BAR_K_FULL + s), kTileBytes);
             tma_load_4d(ctx.sbase + kOffK + s * kTileBytes, &maps.k, ctx.bar(BAR_K_FULL + s), 0,
-                        it.g, kb, it.b);
-            mbar_arrive_expect_tx(ctx.bar(BAR_V_FULL + s), kTileBytes);
-            tma_load_4d(ctx.sbase + kOffV + s * kTileBytes, &maps.v, ctx.bar(BAR_V_FULL + s), 0,
-                        it.g, kb, it.b);
+                        it.g, (it.jt0 + j) * kBlockN, it.b);
             ++G;
           }
         }
         if (*ctx.abort_flag) {
-          // Let every copy this CTA started land before its shared memory is released.
+          // Let every copy this thread started land before shared memory is released.
           volatile int never = 0;
           for (int i = max(0, nq - 2); i < nq; ++i)
             mbar_wait(ctx.bar(BAR_Q_FULL + (i & 1)), (i >> 1) & 1, &never, nullptr, 0,
                       kWaitTimeoutNs);
-          for (int i = max(0, G - kStages); i < G; ++i) {
+          for (int i = max(0, G - kStages); i < G; ++i)
             mbar_wait(ctx.bar(BAR_K_FULL + i % kStages), (i / kStages) & 1, &never, nullptr, 0,
                       kWaitTimeoutNs);
-            mbar_wait(ctx.bar(BAR_V_FULL + i % kStages), (i / kStages) & 1, &never, nullptr, 0,
-                      kWaitTimeoutNs);
-          }
         }
       }
-    } else if (warp == 1) {
-      // -------------------------------------------------------------- MMA issuer
+    } else if (warp == 3) {
+      // -------------------------------------------------------------- V producer
       if (lane == 0 && !skip) {
-        // P.V of tile pv_G (item pv_n) is issued after the next tile's Q.K^T:
-        // the softmax releases S as soon as it has loaded it, long before P.
-        int pv_G = -1, pv_n = 0;
+        prefetch_tensormap(&maps.v);
+        int G = 0, n = 0;
+        Item it;
+        bool ok = true;
+        for (; ok && item_for(args, n, cta, &it); ++n) {
+          for (int j = 0; j < it.n_tiles; ++j) {
+            const int s = G % kStages;
+            if (G >= kStages && !(ok = ctx.wait(BAR_V_EMPTY + s, ((G / kStages) - 1) & 1)))
+              break;
+            mbar_arrive_expect_tx(ctx.bar(BAR_V_FULL + s), kTileBytes);
+            tma_load_4d(ctx.sbase + kOffV + s * kTileBytes, &maps.v, ctx.bar(BAR_V_FULL + s), 0,
+                        it.g, (it.jt0 + j) * kBlockN, it.b);
+            ++G;
+          }
+        }
+        if (*ctx.abort_flag) {
+          volatile int never = 0;
+          for (int i = max(0, G - kStages); i < G; ++i)
+            mbar_wait(ctx.bar(BAR_V_FULL + i % kStages), (i / kStages) & 1, &never, nullptr, 0,
+                      kWaitTimeoutNs);
+        }
+      }
+    } else {
+      // -------------------------------------------------------------- MMA issuer of M tile m
+      const int m = warp - 1;
+      if (lane == 0 && !skip) {
+        // P.V of tile pv_G is issued after the next tile's Q.K^T: the softmax
+        // releases S as soon as it has loaded it, long before P.
+        int pv_G = -1;
         bool pv_first = false, pv_last = false;
         int G = 0, n = 0;
         Item it;
@@ -356,64 +394,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < it.n_tiles; ++j, ++G) {
             const int s = G % kStages;
             if (!(ok = ctx.wait(BAR_K_FULL + s, (G / kStages) & 1))) break;
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-              if (G > 0 && !(ok = ctx.wait(BAR_S_FREE + m, (G - 1) & 1))) break;
-              tc_fence_after_sync();
-              issue_qk(ctx, tmem, m, qs, s);
-              mma_commit(ctx.bar(BAR_S_FULL + m));
-            }
-            if (!ok) break;
-            if (pv_G >= 0 && !(ok = issue_pv_tile(ctx, tmem, pv_G, pv_n, pv_first, pv_last))) break;
+            if (G > 0 && !(ok = ctx.wait(BAR_S_FREE + m, (G - 1) & 1))) break;
+            tc_fence_after_sync();
+            issue_qk(ctx, tmem, m, qs, s);
+            mma_commit(ctx.bar(BAR_S_FULL + m));
+            mma_commit(ctx.bar(BAR_K_EMPTY + s));
+            if (pv_G >= 0 && !(ok = issue_pv(ctx, tmem, m, pv_G, pv_first, pv_last))) break;
             pv_G = G;
-            pv_n = n;
             pv_first = j == 0;
             pv_last = j == it.n_tiles - 1;
           }
         }
-        if (ok && pv_G >= 0) issue_pv_tile(ctx, tmem, pv_G, pv_n, pv_first, pv_last);
+        if (ok && pv_G >= 0) issue_pv(ctx, tmem, m, pv_G, pv_first, pv_last);
         // Every MMA issued must finish before the tensor memory is released.
-        mma_commit(ctx.bar(BAR_MMA_DONE));
+        mma_commit(ctx.bar(BAR_MMA_DONE + m));
         volatile int never = 0;
-        mbar_wait(ctx.bar(BAR_MMA_DONE), 0, &never, nullptr, 0, kWaitTimeoutNs);
-      }
-    } else {
-      // -------------------------------------------------------------- RoPE
-      const int t = static_cast<int>(threadIdx.x) - 64;  // 0..63
-      int n = 0;
-      Item it;
-      bool ok = !skip;
-      for (; ok && item_for(args, n, cta, &it); ++n) {
-        const int qs = n & 1;
-        if (!(ok = ctx.wait_warp(BAR_Q_FULL + qs, (n >> 1) & 1))) break;
-        const float2* tab = reinterpret_cast<const float2*>(smem + kOffTab + qs * kTabSlotBytes);
-#pragma unroll 1
-        for (int i = 0; i < 4; ++i) {
-          const int row = t + 64 * (i & 1);
-          const int tl = (i >> 1) * kTokensPerM + (row >> 3);  // token within the item
-          if (it.q0 + tl < S)
-            rope_row(smem + kOffQ + (2 * qs + (i >> 1)) * kTileBytes + row * 128, row,
-                     tab + tl * kRopePairs);
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(ctx.bar(BAR_Q_READY + qs));
+        mbar_wait(ctx.bar(BAR_MMA_DONE + m), 0, &never, nullptr, 0, kWaitTimeoutNs);
       }
     }
   } else if (wg == 1 || wg == 2) {
-    // ---------------------------------------------------------------- softmax
+    // ---------------------------------------------------------------- softmax + epilogue
     setmaxnreg_inc<kRegsSoftmax>();
     const int m = wg - 1;          // M tile
     const int wq = warp & 3;       // TMEM lane quarter of this warp
     const int r = wq * 32 + lane;  // row of the M tile = TMEM lane
+    const bool elected = wq == 0 && lane == 0;  // issues this warpgroup's output stores
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + tmem_s(m);
     const uint32_t tP = tmem + lane_off + tmem_p(m);
     const uint32_t tO = tmem + lane_off + tmem_o(m);
     int G = 0, n = 0;
+    int store_slot = -1;  // Q slot whose output store may still be reading shared memory
     Item it;
     bool ok = !skip;
     for (; ok && item_for(args, n, cta, &it); ++n) {
+      const int qs = n & 1;
       const int tq = it.q0 + m * kTokensPerM + (r >> 3);
       const int tmin = it.q0 + m * kTokensPerM + wq * 4;  // tokens of this warp: tmin .. tmin+3
       const int tmax = tmin + 3;
@@ -430,6 +445,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(ctx.bar(BAR_S_FREE + m));
+        if (store_slot >= 0 && elected) {
+          // The previous item's output store has long finished reading its
+          // staging tile; hand the Q slot back to the producer.
+          tma_store_wait_read();
+          mbar_arrive(ctx.bar(BAR_Q_EMPTY + store_slot));
+        }
+        store_slot = -1;
         const int kb = (it.jt0 + j) * kBlockN;
         const bool wmask = (kb + kBlockN - 1 > tmin) || (W > 0 && kb <= tmax - W);
         if (wmask) {
@@ -487,16 +509,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc1 = fadd2(acc1, f2_pack(p2, p3));
           sv[i] = pack_bf16x2(p0, p1);
           sv[i + 1] = pack_bf16x2(p2, p3);
+          if (i == kTurnHandOff) {
+            // Hand the exponential unit to the other warpgroup before this
+            // loop ends: its wake-up overlaps these last exponentials.
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ctx.bar(BAR_TURN + (m ^ 1)));
+          }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(ctx.bar(BAR_TURN + (m ^ 1)));
         {
           float a0, a1, a2, a3;
           f2_unpack(acc0, a0, a1);
           f2_unpack(acc1, a2, a3);
           l += (a0 + a1) + (a2 + a3);
         }
-        // P and O are free once the previous tile's P.V has completed.
+        // P is free once the previous tile's P.V has completed.
         if (G > 0 && !(ok = ctx.wait_warp(BAR_P_FREE + m, (G - 1) & 1))) break;
         tc_fence_after_sync();
         {
@@ -521,74 +547,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(ctx.bar(BAR_P_FULL + m));
       }
       if (!ok) break;
-      // hand the row sum to the epilogue
-      if (n >= 1 && !(ok = ctx.wait_warp(BAR_L_EMPTY + m, (n - 1) & 1))) break;
-      l_smem[m * 128 + r] = l;
+      // ---- epilogue: O / l -> bf16 -> this M tile's half of the item's Q slot -> TMA store.
+      // O_FULL follows the item's last P.V, so every Q.K^T that read the Q tile is done too.
+      if (!(ok = ctx.wait_warp(BAR_O_FULL + m, n & 1))) break;
+      tc_fence_after_sync();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      uint8_t* stage = smem + kOffQ + (2 * qs + m) * kTileBytes;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t ov[32];
+        tmem_ld32(tO + 32 * half, ov);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(ov[8 * cc + 2 * e]) * inv_l,
+                               __uint_as_float(ov[8 * cc + 2 * e + 1]) * inv_l);
+          const int chunk = 4 * half + cc;
+          *reinterpret_cast<uint4*>(stage + r * 128 + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      // O has been read: the next item's first P.V (which overwrites it) is
+      // issued only after this warpgroup's next P_FULL.
+      tc_fence_before_sync();
+      fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ctx.bar(BAR_L_FULL + m));
+      if (lane == 0) mbar_arrive(ctx.bar(BAR_STAGED + m));
+      if (elected) {
+        ok = ctx.wait(BAR_STAGED + m, n & 1);
+        if (ok && it.q0 + m * kTokensPerM < S)
+          tma_store_4d(&maps.o, ctx.q_tile(qs, m), 0, it.g * kGroup, it.q0 + m * kTokensPerM,
+                       it.b);
+        tma_store_commit();
+      }
+      store_slot = qs;
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (elected) {
+      tma_store_wait_all();
+      if (ok && store_slot >= 0) mbar_arrive(ctx.bar(BAR_Q_EMPTY + store_slot));
     }
   } else {
-    // ---------------------------------------------------------------- epilogue
+    // ---------------------------------------------------------------- RoPE
     setmaxnreg_dec<kRegsLight>();
-    const int wq = warp & 3;
-    const int r = wq * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const int t = static_cast<int>(threadIdx.x) - 384;  // 0..127: row t of both M tiles
     int n = 0;
     Item it;
-    // Every thread runs every item (no early exit) so the named barrier
-    // below is always reached by all 128 threads; failed waits skip work.
-    for (; item_for(args, n, cta, &it); ++n) {
+    bool ok = !skip;
+    for (; ok && item_for(args, n, cta, &it); ++n) {
       const int qs = n & 1;
-      bool ok = !skip && !*ctx.abort_flag;
+      if (!(ok = ctx.wait_warp(BAR_Q_FULL + qs, (n >> 1) & 1))) break;
+      const uint8_t* tab = smem + kOffTab + qs * kTabSlotBytes;
 #pragma unroll 1
-      for (int m = 0; m < 2; ++m) {
-        const bool ok_o = ok && ctx.wait_warp(BAR_O_FULL + m, n & 1) &&
-                          ctx.wait_warp(BAR_L_FULL + m, n & 1);
-        if (ok_o) {
-          const float inv_l = 1.f / l_smem[m * 128 + r];
-          __syncwarp();
-          if (lane == 0) mbar_arrive(ctx.bar(BAR_L_EMPTY + m));
-          tc_fence_after_sync();
-          uint8_t* stage = smem + kOffQ + (2 * qs + m) * kTileBytes;
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t ov[32];
-            tmem_ld32(tmem + lane_off + tmem_o(m) + 32 * half, ov);
-            if (half == 1) {
-              tc_fence_before_sync();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(ctx.bar(BAR_O_EMPTY + m));
-            }
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              uint32_t w[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                w[e] = pack_bf16x2(__uint_as_float(ov[8 * cc + 2 * e]) * inv_l,
-                                   __uint_as_float(ov[8 * cc + 2 * e + 1]) * inv_l);
-              const int chunk = 4 * half + cc;
-              *reinterpret_cast<uint4*>(stage + r * 128 + ((chunk ^ (r & 7)) << 4)) =
-                  make_uint4(w[0], w[1], w[2], w[3]);
-            }
-          }
-        }
-        ok = ok_o;
+      for (int mm = 0; mm < 2; ++mm) {
+        const int tl = mm * kTokensPerM + (t >> 3);  // token within the item
+        if (it.q0 + tl < S)
+          rope_row(smem + kOffQ + (2 * qs + mm) * kTileBytes + t * 128, t,
+                   reinterpret_cast<const float2*>(tab + tl * kTabRowBytes));
       }
       fence_async_smem();
-      named_barrier(1, 128);
-      if (threadIdx.x == 384) {
-        if (ok && !*ctx.abort_flag) {
-          for (int m = 0; m < 2; ++m)
-            if (it.q0 + m * kTokensPerM < S)
-              tma_store_4d(&maps.o, ctx.q_tile(qs, m), 0, it.g * kGroup, it.q0 + m * kTokensPerM,
-                           it.b);
-          tma_store_commit();
-          tma_store_wait_read();
-        }
-        mbar_arrive(ctx.bar(BAR_Q_EMPTY + qs));
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ctx.bar(BAR_Q_READY + qs));
     }
-    if (threadIdx.x == 384) tma_store_wait_all();
   }
 
   tc_fence_before_sync();
@@ -598,7 +620,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, kTmemCols);
   }
 }
-
 
 // ============================================================================
 // Narrow-band kernel for sliding windows 0 < W <= 128 (the model's W = 128).
@@ -772,7 +793,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(ctx.q(s), &maps.q, ctx.bar(band::BAR_QK_FULL + s), 0, it.g * kGroup, it.q0,
                       it.b);
           tma_load_4d(ctx.k(s), &maps.k_band, ctx.bar(band::BAR_QK_FULL + s), 0, it.g, kb, it.b);
-          stage_rope_rows<band::kTokens>(args, it.b, it.q0, ctx.tab(s),
+          stage_rope_rows<band::kTokens, kRopePairs * 8>(args, it.b, it.q0, ctx.tab(s),
                                          ctx.bar(band::BAR_QK_FULL + s));
           mbar_arrive_expect_tx(ctx.bar(band::BAR_V_FULL + s), band::kKVBytes);
           tma_load_4d(ctx.v(s), &maps.v_band, ctx.bar(band::BAR_V_FULL + s), 0, it.g, kb, it.b);

@@ -5,7 +5,7 @@
 // rope_table_kernel: for every position p < 131072 and pair k < 32 the
 //   (cos, sin) of p * theta^(-2k/64). Angles reach 1.3e5 rad, so they are
 //   formed and reduced in fp64; only the results are stored as fp32.
-// rope_keys_kernel: rotates every key row once per layer into a workspace,
+// rope_rows_kernel: rotates every key row once per layer into a workspace,
 //   so the attention kernels, which read each key tile many times, never
 //   rotate keys. HBM bound: 128 bytes read and written per row.
 #include "internal.h"
@@ -26,19 +26,20 @@ __global__ void rope_table_kernel(float2* __restrict__ table) {
 }
 
 // Four threads per 64-element row; thread c rotates the 16-byte chunks c and
-// c+4 (elements 8c..8c+7 pair with 8c+32..8c+39). Rows are [token][kv head],
-// so the eight rows of a token share one position and one table row.
-__global__ void __launch_bounds__(256) rope_keys_kernel(const uint4* __restrict__ k,
+// c+4 (elements 8c..8c+7 pair with 8c+32..8c+39). Rows are [token][head]
+// with 2^heads_log2 heads per token, which share one position and table row.
+__global__ void __launch_bounds__(256) rope_rows_kernel(const uint4* __restrict__ k,
                                                         const int32_t* __restrict__ pos,
                                                         const float2* __restrict__ table,
                                                         uint4* __restrict__ k_rot,
-                                                        int64_t n_rows, int* err) {
+                                                        int64_t n_rows, int heads_log2,
+                                                        int* err) {
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
        idx < n_rows * 4; idx += stride) {
     const int64_t row = idx >> 2;
     const int c = static_cast<int>(idx & 3);
-    int p = __ldg(pos + (row >> 3));
+    int p = __ldg(pos + (row >> heads_log2));
     if (p < 0 || p >= kMaxPosition) {
       atomicOr(err, kErrPosition);
       p = p < 0 ? 0 : kMaxPosition - 1;
@@ -74,14 +75,17 @@ cudaError_t launch_rope_table(float2* table, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_rope_keys(const void* k, const int32_t* pos, const float2* table, void* k_rot,
-                             int64_t n_tokens, int grid_cap, int* err, cudaStream_t stream) {
-  const int64_t n_rows = n_tokens * kNumKvHeads;
+cudaError_t launch_rope_rows(const void* x, const int32_t* pos, const float2* table, void* x_rot,
+                             int64_t n_tokens, int heads, int grid_cap, int* err,
+                             cudaStream_t stream) {
+  const int heads_log2 = heads == kNumHeads ? 6 : 3;
+  const int64_t n_rows = n_tokens * heads;
   const int64_t threads = n_rows * 4;
   int64_t blocks = (threads + 255) / 256;
   if (blocks > grid_cap) blocks = grid_cap;
-  rope_keys_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      static_cast<const uint4*>(k), pos, table, static_cast<uint4*>(k_rot), n_rows, err);
+  rope_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      static_cast<const uint4*>(x), pos, table, static_cast<uint4*>(x_rot), n_rows, heads_log2,
+      err);
   return cudaGetLastError();
 }
 
