@@ -328,6 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           stage_rope_rows<kBlockQ, kTabRowBytes>(args, it.b, it.q0,
                                                  ctx.sbase + kOffTab + qs * kTabSlotBytes,
                                                  ctx.bar(BAR_Q_FULL + qs));
+          // The rotated keys come from the key-rotation kernel launched just
+          // before this one, which may still be running (the launch overlaps
+          // this kernel's prologue and first Q loads with its tail).
+          if (n == 0) griddep_wait();
           nq = n + 1;
           for (int j = 0; j < it.n_tiles; ++j) {
             const int s = G % kStages;
@@ -792,9 +796,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 band::kQBytes + band::kKVBytes + tab_bytes);
           tma_load_4d(ctx.q(s), &maps.q, ctx.bar(band::BAR_QK_FULL + s), 0, it.g * kGroup, it.q0,
                       it.b);
-          tma_load_4d(ctx.k(s), &maps.k_band, ctx.bar(band::BAR_QK_FULL + s), 0, it.g, kb, it.b);
           stage_rope_rows<band::kTokens, kRopePairs * 8>(args, it.b, it.q0, ctx.tab(s),
-                                         ctx.bar(band::BAR_QK_FULL + s));
+                                                         ctx.bar(band::BAR_QK_FULL + s));
+          // rotated keys: see the same wait in prefill_kernel
+          if (k == 0) griddep_wait();
+          tma_load_4d(ctx.k(s), &maps.k_band, ctx.bar(band::BAR_QK_FULL + s), 0, it.g, kb, it.b);
           mbar_arrive_expect_tx(ctx.bar(band::BAR_V_FULL + s), band::kKVBytes);
           tma_load_4d(ctx.v(s), &maps.v_band, ctx.bar(band::BAR_V_FULL + s), 0, it.g, kb, it.b);
         }
@@ -1020,21 +1026,32 @@ int prefill_items(int batch, int seqlen, int window) {
   return (seqlen + tokens - 1) / tokens * kNumKvHeads * batch;
 }
 
+// Both attention kernels are launched with programmatic stream serialization:
+// they may start while the key-rotation kernel before them finishes, and only
+// the thread that loads rotated keys waits for it (griddep_wait).
 cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream) {
   const int grid = args.n_items < args.grid ? args.n_items : args.grid;
-  if (prefill_uses_band(args.window)) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_band_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(band::kSmemBytes));
-    if (e != cudaSuccess) return e;
-    prefill_band_kernel<<<grid, kThreads, band::kSmemBytes, stream>>>(maps, args);
-    return cudaGetLastError();
-  }
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
+  const bool use_band = prefill_uses_band(args.window);
+  const uint32_t smem_bytes = use_band ? band::kSmemBytes : kSmemBytes;
+  cudaError_t e = use_band ? cudaFuncSetAttribute(prefill_band_kernel,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(smem_bytes))
+                           : cudaFuncSetAttribute(prefill_kernel,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(smem_bytes));
   if (e != cudaSuccess) return e;
-  prefill_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps, args);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return use_band ? cudaLaunchKernelEx(&cfg, prefill_band_kernel, maps, args)
+                  : cudaLaunchKernelEx(&cfg, prefill_kernel, maps, args);
 }
 
 }  // namespace gqa

@@ -34,6 +34,9 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const uint4* __restrict_
                                                         uint4* __restrict__ k_rot,
                                                         int64_t n_rows, int heads_log2,
                                                         int* err) {
+  // The attention kernel that follows may launch now; it waits for this
+  // kernel's writes before it reads them.
+  griddep_launch_dependents();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
        idx < n_rows * 4; idx += stride) {

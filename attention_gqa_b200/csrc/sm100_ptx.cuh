@@ -86,6 +86,16 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization may start while the preceding kernel of its stream still
+// runs; griddep_wait() blocks the calling thread until that kernel has
+// completed and its memory writes are visible. griddep_launch_dependents()
+// lets the next such kernel start early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Per-warpgroup register budget changes (all four warps of the warpgroup execute them).
 template <uint32_t N>
 __device__ __forceinline__ void setmaxnreg_inc() {
