@@ -1,6 +1,7 @@
 """Throughput of the gpt-oss attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload step|tiny256|batch16k|seq128k]
 
 One step is one pass of the whole path over one batch of synthetic inputs:
   * prefill, B=1, S=4096, 64 query / 8 key-value heads, head_dim 64: a
@@ -397,12 +398,180 @@ def run_ours(args, rank: int, world: int):
     return 0
 
 
+# ------------------------------------------------------------------ long prefill workloads
+
+LONG_WORKLOADS = {
+    # name: (config id of the seed recipe, B, S, [(layer, window), ...], description)
+    "tiny256": (1, 1, 256, [(0, 0), (1, 128)],
+                "prefill B=1 S=256 64q/8kv d64, one full-causal layer + one W=128 layer "
+                "(launch-latency bound)"),
+    "batch16k": (3, 4, 16384, [(i, 128 if i % 2 == 0 else 0) for i in range(24)],
+                 "prefill B=4 S=16384 64q/8kv d64, 12 W=128 layers + 12 full-causal layers "
+                 "alternating, each with its own inputs"),
+    "seq128k": (5, 1, 131072, [(0, 0), (1, 128)],
+                "prefill B=1 S=131072 64q/8kv d64, one full-causal layer + one W=128 layer"),
+}
+
+
+def oracle_rows_sample(layers, budget_s: float = 12.0):
+    """Times the fp64 oracle on evenly spaced query rows of the given layers
+    ([(q, k, v, sinks, pos, window) device tensors]); returns (TFLOP/s, s, rows, FLOPs)."""
+    import oracle
+    oracle._load()
+    total_flops, total_s, nrows = 0.0, 0.0, 0
+    per_layer = budget_s / len(layers)
+    for q, k, v, sinks, pos, window in layers:
+        B, S = q.shape[0], q.shape[1]
+        kh = k.double().cpu().numpy()
+        vh = v.double().cpu().numpy()
+        sh = sinks.double().cpu().numpy()
+        ph = pos.cpu().numpy()
+        n = 8
+        while True:
+            toks = np.linspace(0, S - 1, n).astype(np.int64)
+            rows = [(int(i % B), int(t)) for i, t in enumerate(toks)]
+            q_rows = np.stack([q[b, t].double().cpu().numpy() for b, t in rows])
+            t0 = time.perf_counter()
+            oracle.prefill_rows(q_rows, kh, vh, sh, ph, window, rows)
+            dt = time.perf_counter() - t0
+            if dt >= per_layer / 3 or n >= 4096:
+                break
+            n *= 4
+        total_flops += sum(4.0 * D * NQ * (min(t + 1, window) if 0 < window < S else t + 1)
+                           for t in toks)
+        total_s += dt
+        nrows += n
+    return total_flops / total_s / 1e12, total_s, nrows, total_flops
+
+
+def run_long(args, name: str):
+    """One GPU: a step is every layer of the named long workload once (distinct
+    buffers per layer, inputs drawn on the device). Prints one JSON line."""
+    import torch
+
+    import attention_gqa_b200 as gqa
+    from attention_gqa_b200 import build
+    build.build()
+    cfg, B, S, layers, desc = LONG_WORKLOADS[name]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    gqa.init()
+    stream = torch.cuda.current_stream()
+    bufs = []
+    for layer, window in layers:
+        def draw(shape, tid):
+            g = torch.Generator(device=dev)
+            g.manual_seed(0x6A77 ^ (cfg << 24) ^ (layer << 12) ^ tid)
+            return torch.randn(shape, generator=g, device=dev, dtype=torch.float32)
+        bufs.append(dict(
+            q=draw((B, S, NQ, D), 1).to(torch.bfloat16), k=draw((B, S, NKV, D), 2).to(torch.bfloat16),
+            v=draw((B, S, NKV, D), 3).to(torch.bfloat16), sinks=draw((NQ,), 4),
+            pos=torch.arange(S, dtype=torch.int32, device=dev).repeat(B, 1).contiguous(),
+            window=window, out=torch.empty(B, S, NQ, D, dtype=torch.bfloat16, device=dev),
+            ws=torch.empty(gqa.prefill_workspace_bytes(B, S), dtype=torch.uint8, device=dev)))
+    steps = max(1, min(args.steps, 20))
+
+    def step(ev=None):
+        for i, p in enumerate(bufs):
+            if ev is not None:
+                ev[i].record(stream)
+            gqa.prefill(p["q"], p["k"], p["v"], p["sinks"], p["pos"], p["window"], out=p["out"],
+                        workspace=p["ws"])
+        if ev is not None:
+            ev[len(bufs)].record(stream)
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    gqa.check()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(bufs) + 1)]
+              for _ in range(steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        for s_ in range(steps):
+            flush.fill_(s_ & 0xFF)
+            step(events[s_])
+        torch.cuda.synchronize()
+    gqa.check()
+    seg = np.array([[events[s_][i].elapsed_time(events[s_][i + 1]) for i in range(len(bufs))]
+                    for s_ in range(steps)]).sum(axis=0) / steps        # ms per layer
+    flops = [prefill_flops(B, S, w) for _, w in layers]
+    step_ms = float(seg.sum())
+    value = sum(flops) / (step_ms * 1e-3) / 1e12
+    full = [i for i, (_, w) in enumerate(layers) if w <= 0]
+    slid = [i for i, (_, w) in enumerate(layers) if w > 0]
+    full_ms = float(seg[full].sum()) / len(full)
+    slid_ms = float(seg[slid].sum()) / len(slid)
+    full_tf = prefill_flops(B, S, 0) / (full_ms * 1e-3) / 1e12
+    slid_tf = prefill_flops(B, S, 128) / (slid_ms * 1e-3) / 1e12
+    # algorithmic bytes of a sliding layer incl. the key pre-pass (read k, write rotated k)
+    slid_bytes = prefill_bytes(B, S) + 2.0 * B * S * NKV * D * 2
+    hbm, tf_burst, tf_sus, peak_src = load_peaks()
+
+    # end to end through host buffers, one full-causal layer
+    p = bufs[full[0]]
+    hq, hk, hv = (p[n].cpu().pin_memory() for n in ("q", "k", "v"))
+    hs, hp = p["sinks"].cpu().pin_memory(), p["pos"].cpu().pin_memory()
+    ho = torch.empty(p["out"].shape, dtype=torch.bfloat16).pin_memory()
+    gqa.prefill(hq, hk, hv, hs, hp, 0, out=ho)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    gqa.prefill(hq, hk, hv, hs, hp, 0, out=ho)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_tf = prefill_flops(B, S, 0) / (e0.elapsed_time(e1) * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs, hp))
+
+    cpu_v, cpu_s, cpu_rows, cpu_flops = oracle_rows_sample(
+        [(bufs[i]["q"], bufs[i]["k"], bufs[i]["v"], bufs[i]["sinks"], bufs[i]["pos"], layers[i][1])
+         for i in (full[0], slid[0])])
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: N(0,1) bf16 q/k/v and fp32 sinks drawn on the device (torch "
+                "generator seeded per layer), pos = token index",
+        "config": {"workload": desc,
+                   "l2": "flushed before every step (256 MB write)" +
+                         ("; every layer's inputs exceed L2" if prefill_bytes(B, S) > 126e6
+                          else "; a layer's inputs fit in L2"),
+                   "full_layer_ms": full_ms, "full_layer_tflops": full_tf,
+                   "sliding_layer_ms": slid_ms, "sliding_layer_tflops": slid_tf,
+                   "sliding_layer_gbs": slid_bytes / (slid_ms * 1e-3) / 1e9},
+        "roofline": {"kernel": "prefill (key rotation + prefill_kernel, full-causal layer)",
+                     "bound": "tensor", "achieved": full_tf, "peak": tf_sus, "unit": "TFLOP/s",
+                     "frac": full_tf / tf_sus, "peak_source": peak_src + " (sustained)",
+                     "traffic": None, "algorithmic_bytes": prefill_bytes(B, S),
+                     "launch_ms": full_ms},
+        "sliding_roofline": {"bound": "hbm", "achieved": slid_bytes / (slid_ms * 1e-3) / 1e9,
+                             "peak": hbm, "unit": "GB/s",
+                             "frac": slid_bytes / (slid_ms * 1e-3) / 1e9 / hbm},
+        "cpu_baseline": {"value": cpu_v, "unit": "TFLOP/s", "cores": host_cores(),
+                         "kind": "oracle",
+                         "sample": "%d evenly spaced query rows (all 64 heads) of one full and "
+                                   "one sliding layer, %.3g unmasked FLOPs, %.1f s"
+                                   % (cpu_rows, cpu_flops, cpu_s)},
+        "e2e": {"value": e2e_tf, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": ho.numel() * ho.element_size(),
+                "what": "one full-causal layer via host buffers"},
+        "gpu_launches": steps * 2 * len(layers),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["step"] + sorted(LONG_WORKLOADS), default="step",
+                    help="step: the default prefill + decode step; tiny256 / batch16k / "
+                         "seq128k: other prefill workloads (one GPU, at most 20 timed steps)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -410,6 +579,11 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args, rank)
+    if args.workload != "step":
+        if world > 1:
+            print("--workload %s runs on one GPU" % args.workload, file=sys.stderr)
+            return 2
+        return run_long(args, args.workload)
     return run_ours(args, rank, world)
 
 
