@@ -64,6 +64,8 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 
 __global__ void __launch_bounds__(kThreads)
     decode_kernel(const __grid_constant__ DecodeMaps maps, const DecodeArgs a) {
+  // The combine kernel may launch now; it waits for this grid before reading.
+  griddep_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -283,6 +285,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeArgs a) {
   const int wid = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = static_cast<int>(threadIdx.x & 31);
   if (wid >= a.batch * kNumHeads) return;
+  griddep_wait();  // partials of the split kernel launched just before
   const int h = wid % kNumHeads;
   if (*reinterpret_cast<volatile int*>(a.err) & kErrTimeout) return;
   const float sink = __ldg(a.sinks + h);
@@ -341,9 +344,20 @@ cudaError_t launch_decode(const DecodeMaps& maps, const DecodeArgs& a, cudaStrea
   decode_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  // programmatic dependent launch: the combine grid's launch overlaps the
+  // split kernel's tail; its threads wait for the partials (griddep_wait).
   const int warps = a.batch * kNumHeads;
-  combine_kernel<<<(warps * 32 + 255) / 256, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((warps * 32 + 255) / 256));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, a);
 }
 
 }  // namespace gqa
