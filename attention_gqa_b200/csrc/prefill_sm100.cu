@@ -705,24 +705,6 @@ __device__ __forceinline__ bool item_for(const PrefillArgs& a, int k, int cta, I
   return true;
 }
 
-// O (+)= P V for item p (9 MMAs of K = 16 over the 144-key span), then the
-// commits that publish O and release the item's stage.
-__device__ __forceinline__ bool issue_pv(const Ctx& ctx, uint32_t tmem, int p) {
-  constexpr uint32_t idesc_pv = idesc_bf16(128, kHeadDim, true);
-  const int m = p & 1, s = p % kStages;
-  if (!ctx.wait(BAR_V_FULL + s, (p / kStages) & 1)) return false;
-  if (!ctx.wait(BAR_P_FULL + m, (p >> 1) & 1)) return false;
-  if (p >= 2 && !ctx.wait(BAR_O_EMPTY + m, ((p >> 1) - 1) & 1)) return false;
-  tc_fence_after_sync();
-#pragma unroll
-  for (int kk = 0; kk < kSpan / 16; ++kk)
-    mma_bf16_ts(tmem + tmem_o(m), tmem + tmem_s(m) + 8 * kk, sdesc_sw128(ctx.v(s) + 2048 * kk),
-                idesc_pv, kk > 0 ? 1u : 0u);
-  mma_commit(ctx.bar(BAR_O_FULL + m));
-  mma_commit(ctx.bar(BAR_EMPTY + s));
-  return true;
-}
-
 }  // namespace band
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -816,25 +798,69 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 1) {
       // -------------------------------------------------------------- MMA issuer
+      // Q.K^T of item kq and P.V of item kp are independent, so they are issued
+      // in whichever order their inputs arrive (rotated Q for Q.K^T, P for
+      // P.V): a late rotation must not hold back the P.V that frees a stage.
+      // Q.K^T of item kq overwrites S/P of item kq-2, so it is issued only
+      // after that item's P.V (the tensor core runs one thread's MMAs in order).
       if (lane == 0 && !skip) {
         constexpr uint32_t idesc_qk = idesc_bf16(128, band::kSpan, false);
-        int k = 0;
-        band::Item it;
+        constexpr uint32_t idesc_pv = idesc_bf16(128, kHeadDim, true);
+        const int grid = static_cast<int>(gridDim.x);
+        const int n_mine = (args.n_items - cta + grid - 1) / grid;
+        int kq = 0, kp = 0;
         bool ok = true;
-        for (; band::item_for(args, k, cta, &it); ++k) {
-          const int m = k & 1, s = k % band::kStages;
-          if (!(ok = ctx.wait(band::BAR_QK_FULL + s, (k / band::kStages) & 1) &&
-                     ctx.wait(band::BAR_READY + s, (k / band::kStages) & 1)))
-            break;
-          tc_fence_after_sync();
+        uint64_t t_progress = global_timer_ns();
+        uint32_t idle = 0;
+        while (ok && kp < n_mine) {
+          bool progressed = false;
+          if (kq < n_mine && kq <= kp + 1) {
+            const int s = kq % band::kStages, m = kq & 1;
+            const uint32_t ph = (kq / band::kStages) & 1;
+            if (mbar_test_wait(ctx.bar(band::BAR_QK_FULL + s), ph) &&
+                mbar_test_wait(ctx.bar(band::BAR_READY + s), ph)) {
+              tc_fence_after_sync();
 #pragma unroll
-          for (int kk = 0; kk < kHeadDim / 16; ++kk)
-            mma_bf16_ss(tmem + band::tmem_s(m), sdesc_sw128(ctx.q(s) + 32 * kk),
-                        sdesc_sw128(ctx.k(s) + 32 * kk), idesc_qk, kk > 0 ? 1u : 0u);
-          mma_commit(ctx.bar(band::BAR_S_FULL + m));
-          if (k > 0 && !(ok = band::issue_pv(ctx, tmem, k - 1))) break;
+              for (int kk = 0; kk < kHeadDim / 16; ++kk)
+                mma_bf16_ss(tmem + band::tmem_s(m), sdesc_sw128(ctx.q(s) + 32 * kk),
+                            sdesc_sw128(ctx.k(s) + 32 * kk), idesc_qk, kk > 0 ? 1u : 0u);
+              mma_commit(ctx.bar(band::BAR_S_FULL + m));
+              ++kq;
+              progressed = true;
+            }
+          }
+          if (kp < kq) {
+            const int p = kp, m = p & 1, s = p % band::kStages;
+            if (mbar_test_wait(ctx.bar(band::BAR_V_FULL + s), (p / band::kStages) & 1) &&
+                mbar_test_wait(ctx.bar(band::BAR_P_FULL + m), (p >> 1) & 1) &&
+                (p < 2 || mbar_test_wait(ctx.bar(band::BAR_O_EMPTY + m), ((p >> 1) - 1) & 1))) {
+              tc_fence_after_sync();
+#pragma unroll
+              for (int kk = 0; kk < band::kSpan / 16; ++kk)
+                mma_bf16_ts(tmem + band::tmem_o(m), tmem + band::tmem_s(m) + 8 * kk,
+                            sdesc_sw128(ctx.v(s) + 2048 * kk), idesc_pv, kk > 0 ? 1u : 0u);
+              mma_commit(ctx.bar(band::BAR_O_FULL + m));
+              mma_commit(ctx.bar(band::BAR_EMPTY + s));
+              ++kp;
+              progressed = true;
+            }
+          }
+          if (progressed) {
+            idle = 0;
+            t_progress = global_timer_ns();
+          } else {
+            __nanosleep(32);
+            if ((++idle & 63u) == 0u) {
+              if (*ctx.abort_flag) {
+                ok = false;
+              } else if (global_timer_ns() - t_progress > kWaitTimeoutNs) {
+                *ctx.abort_flag = 1;
+                atomicOr(args.err, kErrTimeout);
+                ok = false;
+              }
+            }
+          }
         }
-        if (ok && k > 0) band::issue_pv(ctx, tmem, k - 1);
         mma_commit(ctx.bar(band::BAR_MMA_DONE));
         volatile int never = 0;
         mbar_wait(ctx.bar(band::BAR_MMA_DONE), 0, &never, nullptr, 0, kWaitTimeoutNs);
