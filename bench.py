@@ -221,12 +221,12 @@ def run_ours(args, rank: int, world: int):
 
     import attention_gqa_b200 as gqa
     import synth
+    from attention_gqa_b200 import shard
 
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", device_id=dev)
+    shard.init_from_env("nccl", dev)
     if rank == 0:
         from attention_gqa_b200 import build
         build.build()
@@ -302,10 +302,7 @@ def run_ours(args, rank: int, world: int):
     seg = np.array([[events[s][i].elapsed_time(events[s][i + 1]) for i in range(n_marks - 1)]
                     for s in range(args.steps)])  # ms, [steps, kernels]
     seg_total = seg.sum(axis=0)                                       # ms per segment over K steps
-    if world > 1:
-        t = torch.tensor(seg_total, dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        seg_total = t.cpu().numpy()
+    seg_total = np.array(shard.max_over_ranks(seg_total, dev))  # the slowest rank sets the time
     npre = len(PREFILL_LAYERS)
     pre_ms = float(seg_total[:npre].sum()) / args.steps
     dec_ms = float(seg_total[npre:].sum()) / args.steps
@@ -351,10 +348,7 @@ def run_ours(args, rank: int, world: int):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = shard.max_over_ranks([e2e_ms], dev)[0]
     e2e_value = world * pre_flops / (e2e_ms * 1e-3) / 1e12
 
     if rank == 0:
