@@ -21,7 +21,7 @@ import os
 import torch
 
 __all__ = ["prefill", "decode", "decode_noalloc", "prefill_workspace_bytes",
-           "decode_workspace_bytes", "check", "init", "rope_table",
+           "decode_workspace_bytes", "check", "debug_wait_timeout", "init", "rope_table",
            "library_path", "GptossAttnError", "NUM_HEADS", "NUM_KV_HEADS", "HEAD_DIM",
            "MAX_POSITION"]
 
@@ -73,6 +73,8 @@ def _load():
     lib.gptoss_attn_decode.restype = i32
     lib.gptoss_attn_check.argtypes = [vp]
     lib.gptoss_attn_check.restype = i32
+    lib.gptoss_attn_debug_wait_timeout.argtypes = [ctypes.c_uint, vp]
+    lib.gptoss_attn_debug_wait_timeout.restype = i32
     if lib.gptoss_attn_abi_version() != ABI_VERSION:
         raise ImportError("%s has ABI %d, expected %d" % (path, lib.gptoss_attn_abi_version(),
                                                           ABI_VERSION))
@@ -274,3 +276,10 @@ def decode_noalloc(q, kcache, vcache, sinks, lengths, window: int = 0, out=None,
 def check(stream=None) -> None:
     """Synchronize and raise if a kernel reported a device-side error."""
     _raise(_load().gptoss_attn_check(_stream_handle(stream)), "gptoss_attn_check")
+
+
+def debug_wait_timeout(timeout_us: int, stream=None) -> None:
+    """Diagnostic: run the bounded pipeline wait against a barrier that never
+    completes; the next check() raises the device-timeout status."""
+    _raise(_load().gptoss_attn_debug_wait_timeout(int(timeout_us), _stream_handle(stream)),
+           "gptoss_attn_debug_wait_timeout")

@@ -220,6 +220,18 @@ int gptoss_attn_decode(const void* q, const void* kcache, const void* vcache, co
   return launch_decode(maps, a, stream) == cudaSuccess ? GPTOSS_ATTN_OK : GPTOSS_ATTN_ERR_LAUNCH;
 }
 
+int gptoss_attn_debug_wait_timeout(unsigned timeout_us, cudaStream_t stream) {
+  if (timeout_us == 0 || timeout_us > 2000000u) return GPTOSS_ATTN_ERR_BAD_SHAPE;
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, false);
+  if (st != GPTOSS_ATTN_OK) return st;
+  return launch_wait_timeout(g_state[dev].err, static_cast<uint64_t>(timeout_us) * 1000u,
+                             stream) == cudaSuccess
+             ? GPTOSS_ATTN_OK
+             : GPTOSS_ATTN_ERR_LAUNCH;
+}
+
 int gptoss_attn_check(cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)

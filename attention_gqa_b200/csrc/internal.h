@@ -50,6 +50,9 @@ int prefill_items(int batch, int seqlen, int window);
 // Launches the prefill kernel; returns a cudaError_t.
 cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream);
 
+// Diagnostic: a bounded wait on a barrier nothing arrives at (sets kErrTimeout).
+cudaError_t launch_wait_timeout(int* err, uint64_t timeout_ns, cudaStream_t stream);
+
 // Fills the rotary table [kMaxPosition][32] of (cos, sin).
 cudaError_t launch_rope_table(float2* table, cudaStream_t stream);
 

@@ -70,7 +70,28 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const uint4* __restrict_
   }
 }
 
+// Diagnostic: one thread waits, with the library's bounded wait, on an
+// mbarrier that nothing ever arrives at; when the limit runs out the wait
+// raises the timeout bit of the error word and the kernel returns.
+__global__ void wait_timeout_kernel(int* err, uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    mbar_wait(smem_u32(&bar), 0, &abort_flag, err, kErrTimeout, timeout_ns);
+}
+
 }  // namespace
+
+cudaError_t launch_wait_timeout(int* err, uint64_t timeout_ns, cudaStream_t stream) {
+  wait_timeout_kernel<<<1, 32, 0, stream>>>(err, timeout_ns);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_rope_table(float2* table, cudaStream_t stream) {
   const int n = kMaxPosition * kRopePairs;

@@ -182,6 +182,18 @@ int gptoss_attn_decode_noalloc(const void* q, const void* kcache, const void* vc
                                int batch, int max_len, cudaStream_t stream);
 
 /*
+ * Diagnostic, with no counterpart on the gpt-oss pages: exercises the failure
+ * path every kernel pipeline wait uses. One thread waits, through the same
+ * bounded wait, on a barrier that nothing arrives at; after timeout_us
+ * microseconds (1 .. 2000000, else GPTOSS_ATTN_ERR_BAD_SHAPE) the wait gives
+ * up, sets the timeout bit of the device error word and the kernel returns, so
+ * the context stays usable. Until gptoss_attn_check() clears the word,
+ * prefill and decode kernels launched on this device skip their work; check
+ * then reports GPTOSS_ATTN_ERR_DEVICE_TIMEOUT. Asynchronous on `stream`.
+ */
+int gptoss_attn_debug_wait_timeout(unsigned timeout_us, cudaStream_t stream);
+
+/*
  * Synchronizes `stream`, then reads and clears the current device's error
  * word. Returns GPTOSS_ATTN_OK, GPTOSS_ATTN_ERR_DEVICE_TIMEOUT,
  * GPTOSS_ATTN_ERR_BAD_POSITION, GPTOSS_ATTN_ERR_BAD_LENGTH or

@@ -115,3 +115,9 @@ def test_python_binding_refuses_without_device():
     kv = torch.zeros(1, 4, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(RuntimeError):
         gqa.prefill(q, kv, kv, torch.zeros(64), torch.zeros(1, 4, dtype=torch.int32), 0)
+
+
+def test_debug_wait_timeout_argument_errors(lib):
+    c = _header_codes()
+    assert lib.gptoss_attn_debug_wait_timeout(0, None) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert lib.gptoss_attn_debug_wait_timeout(2000001, None) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
