@@ -21,7 +21,7 @@ import os
 import torch
 
 __all__ = ["prefill", "decode", "decode_noalloc", "prefill_workspace_bytes",
-           "decode_workspace_bytes", "check", "debug_wait_timeout", "init", "rope_table",
+           "decode_workspace_bytes", "prefill_chunk", "check", "debug_wait_timeout", "init", "rope_table",
            "library_path", "GptossAttnError", "NUM_HEADS", "NUM_KV_HEADS", "HEAD_DIM",
            "MAX_POSITION"]
 
@@ -67,6 +67,9 @@ def _load():
     lib.gptoss_attn_prefill_workspace_bytes.restype = sz
     lib.gptoss_attn_prefill.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, vp, sz, vp]
     lib.gptoss_attn_prefill.restype = i32
+    lib.gptoss_attn_prefill_chunk.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32,
+                                              i32, vp]
+    lib.gptoss_attn_prefill_chunk.restype = i32
     lib.gptoss_attn_decode_workspace_bytes.argtypes = [i32, i32, i32]
     lib.gptoss_attn_decode_workspace_bytes.restype = sz
     lib.gptoss_attn_decode.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, vp, sz, vp]
@@ -192,6 +195,43 @@ def prefill(q, k, v, sinks, pos, window: int = 0, out=None, workspace=None,
                                  workspace.numel() * workspace.element_size(),
                                  _stream_handle(stream))
     _raise(st, "gptoss_attn_prefill")
+    return dev_out
+
+
+def prefill_chunk(q, k, v, sinks, pos, kcache, vcache, start: int, window: int = 0, out=None,
+                  stream=None) -> torch.Tensor:
+    """Prefill of the next n = q.shape[1] tokens after `start` cached ones: writes
+    their rotated keys and values into rows [start, start+n) of kcache / vcache
+    ([B, max_len, 8, 64], device) and returns the chunk's attention output."""
+    lib = _load()
+    device = _target_device(q, k, v)
+    q = _dev(q, torch.bfloat16, "q", device)
+    k = _dev(k, torch.bfloat16, "k", device)
+    v = _dev(v, torch.bfloat16, "v", device)
+    sinks = _dev(sinks, torch.float32, "sinks", device)
+    pos = _dev(pos, torch.int32, "pos", device)
+    for name, t in (("kcache", kcache), ("vcache", vcache)):
+        if t.device != device or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous bf16 tensor on %s" % (name, device))
+    if q.dim() != 4 or q.shape[2:] != (NUM_HEADS, HEAD_DIM):
+        raise ValueError("q must be [B, n, 64, 64], got %s" % (tuple(q.shape),))
+    B, n = q.shape[0], q.shape[1]
+    for name, t in (("k", k), ("v", v)):
+        if tuple(t.shape) != (B, n, NUM_KV_HEADS, HEAD_DIM):
+            raise ValueError("%s must be [B, n, 8, 64], got %s" % (name, tuple(t.shape)))
+    if kcache.dim() != 4 or kcache.shape[0] != B or kcache.shape[2:] != (NUM_KV_HEADS, HEAD_DIM):
+        raise ValueError("kcache must be [B, max_len, 8, 64]")
+    if vcache.shape != kcache.shape:
+        raise ValueError("vcache must match kcache")
+    if tuple(sinks.shape) != (NUM_HEADS,) or tuple(pos.shape) != (B, n):
+        raise ValueError("sinks must be [64] and pos [B, n]")
+    dev_out = out if out is not None else torch.empty((B, n, NUM_HEADS, HEAD_DIM),
+                                                      dtype=torch.bfloat16, device=device)
+    st = lib.gptoss_attn_prefill_chunk(q.data_ptr(), k.data_ptr(), v.data_ptr(), sinks.data_ptr(),
+                                       pos.data_ptr(), int(window), dev_out.data_ptr(),
+                                       kcache.data_ptr(), vcache.data_ptr(), B, int(start), n,
+                                       kcache.shape[1], _stream_handle(stream))
+    _raise(st, "gptoss_attn_prefill_chunk")
     return dev_out
 
 

@@ -153,13 +153,82 @@ int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float
   args.err = g_state[dev].err;
   args.batch = batch;
   args.seqlen = seqlen;
+  args.q_start = 0;
   // A window covering the whole sequence is full causal.
   args.window = (window > 0 && window < seqlen) ? window : 0;
   args.n_qtiles = (seqlen + 31) / 32;
   args.n_items = prefill_items(batch, seqlen, args.window);
   args.grid = g_state[dev].num_sms;
-  if (launch_rope_rows(k, pos, args.rope, workspace, static_cast<int64_t>(batch) * seqlen,
-                       kNumKvHeads, args.grid * 8, args.err, stream) != cudaSuccess)
+  if (launch_rope_rows(k, pos, args.rope, workspace, batch, seqlen, seqlen, 0, kNumKvHeads,
+                       args.grid * 8, args.err, stream) != cudaSuccess)
+    return GPTOSS_ATTN_ERR_LAUNCH;
+  return launch_prefill(maps, args, stream) == cudaSuccess ? GPTOSS_ATTN_OK
+                                                           : GPTOSS_ATTN_ERR_LAUNCH;
+}
+
+int gptoss_attn_prefill_chunk(const void* q, const void* k, const void* v, const float* sinks,
+                              const int32_t* pos, int window, void* out, void* kcache,
+                              void* vcache, int batch, int start, int n, int max_len,
+                              cudaStream_t stream) {
+  if (!q || !k || !v || !sinks || !pos || !out || !kcache || !vcache)
+    return GPTOSS_ATTN_ERR_NULL_PTR;
+  if (batch < 1 || batch > 65535 || n < 1 || start < 0 || max_len > kMaxPosition ||
+      static_cast<int64_t>(start) + n > max_len)
+    return GPTOSS_ATTN_ERR_BAD_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kcache) ||
+      !aligned16(vcache) || (reinterpret_cast<uintptr_t>(sinks) & 3u) ||
+      (reinterpret_cast<uintptr_t>(pos) & 3u))
+    return GPTOSS_ATTN_ERR_BAD_ALIGN;
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, true);
+  if (st != GPTOSS_ATTN_OK) return st;
+
+  const int keys = start + n;  // keys visible to the chunk: the cached prefix and the chunk
+  PrefillMaps maps;
+  const uint64_t N = static_cast<uint64_t>(n), B = static_cast<uint64_t>(batch);
+  const uint64_t L = static_cast<uint64_t>(max_len);
+  const uint64_t qdims[4] = {kHeadDim, kNumHeads, N, B};
+  const uint64_t qstr[3] = {kHeadDim * 2, kNumHeads * kHeadDim * 2, N * kNumHeads * kHeadDim * 2};
+  const uint32_t qbox[4] = {kHeadDim, kGroup, 16, 1};
+  // cache views end at the chunk's last key, so the tensor memory engine
+  // zero-fills (never reads) cache rows past it
+  const uint64_t cdims[4] = {kHeadDim, kNumKvHeads, static_cast<uint64_t>(keys), B};
+  const uint64_t cstr[3] = {kHeadDim * 2, kNumKvHeads * kHeadDim * 2,
+                            L * kNumKvHeads * kHeadDim * 2};
+  const uint32_t kbox[4] = {kHeadDim, 1, 128, 1};
+  const uint32_t kbox_band[4] = {kHeadDim, 1, 144, 1};
+  if (!make_tmap_bf16_4d(&maps.q, q, qdims, qstr, qbox) ||
+      !make_tmap_bf16_4d(&maps.o, out, qdims, qstr, qbox) ||
+      !make_tmap_bf16_4d(&maps.k, kcache, cdims, cstr, kbox) ||
+      !make_tmap_bf16_4d(&maps.v, vcache, cdims, cstr, kbox) ||
+      !make_tmap_bf16_4d(&maps.k_band, kcache, cdims, cstr, kbox_band) ||
+      !make_tmap_bf16_4d(&maps.v_band, vcache, cdims, cstr, kbox_band))
+    return GPTOSS_ATTN_ERR_TENSOR_MAP;
+
+  PrefillArgs args;
+  args.pos = pos;
+  args.sinks = sinks;
+  args.rope = g_state[dev].rope;
+  args.err = g_state[dev].err;
+  args.batch = batch;
+  args.seqlen = n;
+  args.q_start = start;
+  // A window covering every visible key is full causal.
+  args.window = (window > 0 && window < keys) ? window : 0;
+  args.n_qtiles = (n + 31) / 32;
+  args.n_items = prefill_items(batch, n, args.window);
+  args.grid = g_state[dev].num_sms;
+  // values into the cache, then the rotated keys, then the attention (which
+  // may start during the key rotation and waits for it before reading keys)
+  const size_t row = static_cast<size_t>(kNumKvHeads) * kHeadDim * 2;
+  if (cudaMemcpy2DAsync(static_cast<uint8_t*>(vcache) + static_cast<size_t>(start) * row,
+                        static_cast<size_t>(max_len) * row, v, static_cast<size_t>(n) * row,
+                        static_cast<size_t>(n) * row, static_cast<size_t>(batch),
+                        cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+    return GPTOSS_ATTN_ERR_LAUNCH;
+  if (launch_rope_rows(k, pos, args.rope, kcache, batch, n, max_len, start, kNumKvHeads,
+                       args.grid * 8, args.err, stream) != cudaSuccess)
     return GPTOSS_ATTN_ERR_LAUNCH;
   return launch_prefill(maps, args, stream) == cudaSuccess ? GPTOSS_ATTN_OK
                                                            : GPTOSS_ATTN_ERR_LAUNCH;

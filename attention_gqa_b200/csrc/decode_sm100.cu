@@ -221,6 +221,21 @@ __global__ void __launch_bounds__(kThreads)
     const float p10 = ex2_approx(x[1][0] - mr), p11 = ex2_approx(x[1][1] - mr);
     l_part += (p00 + p01) + (p10 + p11);
     const uint32_t pa0 = pack_bf16x2(p00, p01), pa2 = pack_bf16x2(p10, p11);
+    // Keys past the end of the sequence have p = 0, but their cache rows may
+    // hold anything (never written), and 0 * NaN or 0 * Inf would poison O:
+    // zero this warp's V rows of such keys before P.V reads them.
+    const bool tail = key0 + 16 > k_end;
+    if (tail) {
+#pragma unroll
+      for (int c = lane; c < 16 * 8; c += 32) {
+        const int rr = c >> 3;
+        if (key0 + rr >= k_end) {
+          const uint32_t addr = sv + (16 * warp + rr) * 128 + (c & 7) * 16;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+        }
+      }
+      __syncwarp();
+    }
     {
       const int j = lane >> 3, row = lane & 7;
       const int kl = 16 * warp + 8 * (j & 1) + row;
@@ -233,6 +248,9 @@ __global__ void __launch_bounds__(kThreads)
         mma_16816(o[2 * dn + 1], pa0, pa2, b2, b3);
       }
     }
+    // the zeroing above wrote the stage through the generic proxy; order it
+    // before the next TMA write into this stage
+    if (tail) fence_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar(s));
   }

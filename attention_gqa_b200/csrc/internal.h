@@ -30,7 +30,9 @@ struct PrefillArgs {
   const float2* rope;   // [kMaxPosition][32] (cos, sin)
   int* err;             // device error word
   int batch;
-  int seqlen;
+  int seqlen;           // query tokens per sequence (the rows of q, pos and out)
+  int q_start;          // key index of query token 0: keys come from a cache
+                        // whose rows [0, q_start) precede this call's tokens
   int window;           // <= 0: full causal
   int n_qtiles;         // ceil(seqlen / 32)
   int n_items;          // work items (prefill_items)
@@ -56,11 +58,12 @@ cudaError_t launch_wait_timeout(int* err, uint64_t timeout_ns, cudaStream_t stre
 // Fills the rotary table [kMaxPosition][32] of (cos, sin).
 cudaError_t launch_rope_table(float2* table, cudaStream_t stream);
 
-// Rotates the rows of x [n_tokens][heads][64] (bf16; heads = 8 for keys or 64
-// for queries) by pos[token] into x_rot.
+// Rotates the rows of x [batch][n][heads][64] (bf16; heads = 8 for keys or 64
+// for queries) by pos[batch][n] into x_rot laid out [batch][dst_len][heads][64],
+// token t of each sequence going to token dst_start + t.
 cudaError_t launch_rope_rows(const void* x, const int32_t* pos, const float2* table, void* x_rot,
-                             int64_t n_tokens, int heads, int grid_cap, int* err,
-                             cudaStream_t stream);
+                             int batch, int64_t n, int64_t dst_len, int64_t dst_start, int heads,
+                             int grid_cap, int* err, cudaStream_t stream);
 
 struct DecodeArgs {
   const uint16_t* q;       // [B][64][64] bf16, un-rotated

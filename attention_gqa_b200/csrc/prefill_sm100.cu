@@ -138,8 +138,10 @@ __device__ __forceinline__ bool item_for(const PrefillArgs& a, int k, int cta, I
   it->g = rem % kNumKvHeads;
   it->b = rem / kNumKvHeads;
   it->q0 = qt * kBlockQ;
-  const int qlast = min(it->q0 + kBlockQ - 1, a.seqlen - 1);
-  const int klo = a.window > 0 ? max(0, it->q0 - a.window + 1) : 0;
+  // key index of the item's first and last query token
+  const int kq0 = a.q_start + it->q0;
+  const int qlast = a.q_start + min(it->q0 + kBlockQ - 1, a.seqlen - 1);
+  const int klo = a.window > 0 ? max(0, kq0 - a.window + 1) : 0;
   it->jt0 = klo / kBlockN;
   it->n_tiles = qlast / kBlockN - it->jt0 + 1;
   return true;
@@ -433,8 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = !skip;
     for (; ok && item_for(args, n, cta, &it); ++n) {
       const int qs = n & 1;
-      const int tq = it.q0 + m * kTokensPerM + (r >> 3);
-      const int tmin = it.q0 + m * kTokensPerM + wq * 4;  // tokens of this warp: tmin .. tmin+3
+      // key index of this row's query token; this warp's tokens are tmin .. tmin+3
+      const int tq = args.q_start + it.q0 + m * kTokensPerM + (r >> 3);
+      const int tmin = args.q_start + it.q0 + m * kTokensPerM + wq * 4;
       const int tmax = tmin + 3;
       const float sink = __ldg(args.sinks + it.g * kGroup + (r & 7));
       const bool sink_off = isinf(sink) && sink < 0.f;
@@ -643,6 +646,11 @@ constexpr int kTokens = 16;
 constexpr int kSpan = 144;  // 128 keys before the tile + the tile's 16
 constexpr int kStages = 3;
 constexpr int kOutSlots = 3;  // output staging ring; a slot is reused 3 items later
+// Register budgets after the warpgroup split (launch is 512 x 128): the
+// softmax rows here are 144 scores wide, so it gets more than in prefill_kernel.
+constexpr uint32_t kRegsLight = 64;     // WG0 and WG3
+constexpr uint32_t kRegsSoftmax = 192;  // WG1 and WG2
+static_assert(2 * 128 * kRegsLight + 2 * 128 * kRegsSoftmax <= 512 * 128, "register split");
 constexpr uint32_t kQBytes = 128 * 128;
 constexpr uint32_t kKVBytes = kSpan * 128;
 constexpr uint32_t kTabBytes = kTokens * kRopePairs * 8;  // table rows of the 16 tokens
@@ -757,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int wg = warp >> 2;
 
   if (wg == 0) {
-    setmaxnreg_dec<kRegsLight>();
+    setmaxnreg_dec<band::kRegsLight>();
     if (warp == 0) {
       // -------------------------------------------------------------- producer
       if (lane == 0 && !skip) {
@@ -771,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (k >= band::kStages &&
               !ctx.wait(band::BAR_EMPTY + s, ((k / band::kStages) - 1) & 1))
             break;
-          const int kb = it.q0 - 128;
+          const int kb = args.q_start + it.q0 - 128;  // span start, as a key index
           const uint32_t tab_bytes =
               kRopePairs * 8 * static_cast<uint32_t>(min(band::kTokens, S - it.q0));
           mbar_arrive_expect_tx(ctx.bar(band::BAR_QK_FULL + s),
@@ -888,7 +896,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (wg == 1 || wg == 2) {
     // ---------------------------------------------------------------- softmax
-    setmaxnreg_inc<kRegsSoftmax>();
+    setmaxnreg_inc<band::kRegsSoftmax>();
     const int m = wg - 1;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
@@ -897,10 +905,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     band::Item it;
     bool ok = !skip;
     for (int k = m, i = 0; ok && band::item_for(args, k, cta, &it); k += 2, ++i) {
-      // row token q0 + d sees keys (q0+d-W, q0+d], i.e. span columns
-      // [max(128-q0, d+129-W), d+128] of the span starting at key q0-128
+      // row token q0 + d (key index kq0 + d) sees keys (kq0+d-W, kq0+d], i.e.
+      // span columns [max(128-kq0, d+129-W), d+128] of the span starting at
+      // key kq0-128
       const int d = r >> 3;
-      const int c_lo = max(128 - it.q0, d + 129 - W);
+      const int kq0 = args.q_start + it.q0;  // key index of the item's first query token
+      const int c_lo = max(128 - kq0, d + 129 - W);
       const int c_hi = d + 128;
       const float sink = __ldg(args.sinks + it.g * kGroup + (r & 7));
       const bool sink_off = isinf(sink) && sink < 0.f;
@@ -912,7 +922,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // W = 128 and q0 >= 128 that is only [0, 17) and [128, 144).
       // (Only the executed branch occupies the instruction cache, so the
       // common case stays short.)
-      if (W == 128 && it.q0 >= 128) {
+      if (W == 128 && kq0 >= 128) {
 #pragma unroll
         for (int c = 0; c < 17; ++c)
           if (c < c_lo) sv[c] = __float_as_uint(-INFINITY);
@@ -984,7 +994,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- epilogue
-    setmaxnreg_dec<kRegsLight>();
+    setmaxnreg_dec<band::kRegsLight>();
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;

@@ -28,12 +28,16 @@ __global__ void rope_table_kernel(float2* __restrict__ table) {
 // Four threads per 64-element row; thread c rotates the 16-byte chunks c and
 // c+4 (elements 8c..8c+7 pair with 8c+32..8c+39). Rows are [token][head]
 // with 2^heads_log2 heads per token, which share one position and table row.
+// Source tokens are [batch][n]; token t of sequence b is written to token
+// dst_start + t of a destination laid out [batch][dst_len] (a cache), which
+// is the same layout when dst_len == n and dst_start == 0.
 __global__ void __launch_bounds__(256) rope_rows_kernel(const uint4* __restrict__ k,
                                                         const int32_t* __restrict__ pos,
                                                         const float2* __restrict__ table,
                                                         uint4* __restrict__ k_rot,
                                                         int64_t n_rows, int heads_log2,
-                                                        int* err) {
+                                                        int64_t n, int64_t dst_len,
+                                                        int64_t dst_start, int* err) {
   // The attention kernel that follows may launch now; it waits for this
   // kernel's writes before it reads them.
   griddep_launch_dependents();
@@ -42,7 +46,10 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const uint4* __restrict_
        idx < n_rows * 4; idx += stride) {
     const int64_t row = idx >> 2;
     const int c = static_cast<int>(idx & 3);
-    int p = __ldg(pos + (row >> heads_log2));
+    const int64_t tok = row >> heads_log2;
+    const int64_t dst_tok = dst_len == n ? tok + dst_start : tok + (tok / n) * (dst_len - n) + dst_start;
+    const int64_t dst_row = (dst_tok << heads_log2) | (row & ((int64_t{1} << heads_log2) - 1));
+    int p = __ldg(pos + tok);
     if (p < 0 || p >= kMaxPosition) {
       atomicOr(err, kErrPosition);
       p = p < 0 ? 0 : kMaxPosition - 1;
@@ -65,8 +72,8 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const uint4* __restrict_
       ya[e] = pack_bf16x2(fmaf(x1l, cl, -x2l * sl), fmaf(x1h, ch, -x2h * sh));
       yh[e] = pack_bf16x2(fmaf(x2l, cl, x1l * sl), fmaf(x2h, ch, x1h * sh));
     }
-    k_rot[row * 8 + c] = make_uint4(ya[0], ya[1], ya[2], ya[3]);
-    k_rot[row * 8 + c + 4] = make_uint4(yh[0], yh[1], yh[2], yh[3]);
+    k_rot[dst_row * 8 + c] = make_uint4(ya[0], ya[1], ya[2], ya[3]);
+    k_rot[dst_row * 8 + c + 4] = make_uint4(yh[0], yh[1], yh[2], yh[3]);
   }
 }
 
@@ -100,16 +107,16 @@ cudaError_t launch_rope_table(float2* table, cudaStream_t stream) {
 }
 
 cudaError_t launch_rope_rows(const void* x, const int32_t* pos, const float2* table, void* x_rot,
-                             int64_t n_tokens, int heads, int grid_cap, int* err,
-                             cudaStream_t stream) {
+                             int batch, int64_t n, int64_t dst_len, int64_t dst_start, int heads,
+                             int grid_cap, int* err, cudaStream_t stream) {
   const int heads_log2 = heads == kNumHeads ? 6 : 3;
-  const int64_t n_rows = n_tokens * heads;
+  const int64_t n_rows = static_cast<int64_t>(batch) * n * heads;
   const int64_t threads = n_rows * 4;
   int64_t blocks = (threads + 255) / 256;
   if (blocks > grid_cap) blocks = grid_cap;
   rope_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      static_cast<const uint4*>(x), pos, table, static_cast<uint4*>(x_rot), n_rows, heads_log2,
-      err);
+      static_cast<const uint4*>(x), pos, table, static_cast<uint4*>(x_rot), n_rows, heads_log2, n,
+      dst_len, dst_start, err);
   return cudaGetLastError();
 }
 

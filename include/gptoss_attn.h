@@ -124,6 +124,33 @@ int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float
                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Chunked prefill: the next n tokens of sequences whose first `start` tokens
+ * are already in a key/value cache (a prompt prefilled in pieces, or several
+ * new tokens at once against a cache). The same operation as
+ * gptoss_attn_prefill() with query token i of the chunk at key index start+i:
+ * it sees cache keys j <= start+i (and, for W > 0, j > start+i-W). The gpt-oss
+ * pages name the cache (use_cache in the configuration table) but no chunked
+ * step; this is the plainest joining of the prefill and decode operations.
+ *   q       bf16 [batch][n][64][64], not rotated
+ *   k, v    bf16 [batch][n][8][64], the chunk's keys (not rotated) and values
+ *   sinks   fp32 [64]; pos int32 [batch][n], rotary positions of the chunk
+ *   window  <= 0 full causal; W > 0 as above (W >= start+n is full causal)
+ *   out     bf16 [batch][n][64][64]
+ *   kcache, vcache  bf16 [batch][max_len][8][64]: rows [0, start) hold the
+ *           cached keys (already rotated, as gptoss_attn_decode() expects) and
+ *           values; the call writes the chunk's rotated keys to rows
+ *           [start, start+n) of kcache and its values to the same rows of
+ *           vcache, and reads no row at or past start+n
+ *   0 <= start, 1 <= n, start + n <= max_len <= 131072, 1 <= batch <= 65535
+ * No workspace. Kernels on `stream`: the value copy, the key rotation into the
+ * cache, the attention. Calls on the same cache must be serialized.
+ */
+int gptoss_attn_prefill_chunk(const void* q, const void* k, const void* v, const float* sinks,
+                              const int32_t* pos, int window, void* out, void* kcache,
+                              void* vcache, int batch, int start, int n, int max_len,
+                              cudaStream_t stream);
+
+/*
  * Bytes of device workspace gptoss_attn_decode() needs for these sizes.
  * Returns 0 for invalid sizes.
  */

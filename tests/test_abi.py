@@ -121,3 +121,24 @@ def test_debug_wait_timeout_argument_errors(lib):
     c = _header_codes()
     assert lib.gptoss_attn_debug_wait_timeout(0, None) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
     assert lib.gptoss_attn_debug_wait_timeout(2000001, None) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+
+
+def test_prefill_chunk_argument_errors(lib):
+    c = _header_codes()
+    f = lib.gptoss_attn_prefill_chunk
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] + [ctypes.c_void_p] * 3 + \
+        [ctypes.c_int] * 4 + [ctypes.c_void_p]
+    ok = dict(q=16, k=32, v=48, s=64, p=80, w=0, o=96, kc=112, vc=128, b=1, st=0, n=8, L=64)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["q"], a["k"], a["v"], a["s"], a["p"], a["w"], a["o"], a["kc"], a["vc"], a["b"],
+                 a["st"], a["n"], a["L"], None)
+    assert call(kc=None) == c["GPTOSS_ATTN_ERR_NULL_PTR"]
+    assert call(n=0) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert call(st=-1) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert call(st=60) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]          # start + n > max_len
+    assert call(L=131073, n=8) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert call(b=0) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert call(vc=136) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
+    assert call(p=82) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]

@@ -109,3 +109,21 @@ def test_workspace_canaries(cuda_device):
     assert torch.all(ws[:4096] == 0x5A) and torch.all(ws[4096 + need:] == 0x5A)
     assert torch.all(out_buf[:1024] == 2.5) and torch.all(out_buf[1024 + 3 * NQ * D:] == 2.5)
     compare(dev_to_f64(out), _oracle(x, 0), "canaries")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("window", [0, 128])
+def test_cache_rows_past_length_are_never_used(cuda_device, window):
+    """Rows at or past len[b] may hold anything (here NaN): the output must not see them."""
+    lens = [8192, 8000, 4001, 129, 77, 1, 0]
+    x = synth.make_decode_inputs(4, 7, len(lens), 8192, lengths=lens)
+    kb, vb = x["kcache"].copy(), x["vcache"].copy()
+    for b, n in enumerate(lens):
+        kb[b, n:] = 0x7FC0  # bf16 NaN
+        vb[b, n:] = 0x7FC0
+    out = gqa.decode(bits_to_dev(x["q"]), bits_to_dev(kb), bits_to_dev(vb),
+                     torch.from_numpy(x["sinks"]).cuda(), torch.from_numpy(x["len"]).cuda(), window)
+    gqa.check()
+    ref = oracle.decode(synth.bf16_bits_to_f64(x["q"]), synth.bf16_bits_to_f64(x["kcache"]),
+                        synth.bf16_bits_to_f64(x["vcache"]), x["sinks"], x["len"], window)
+    compare(dev_to_f64(out), ref, "decode with NaN past len, W=%d" % window)
