@@ -1,7 +1,7 @@
 """Throughput of the gpt-oss attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload step|tiny256|batch16k|seq128k]
+                    [--workload step|tiny256|batch16k|seq128k|chunk16k]
 
 One step is one pass of the whole path over one batch of synthetic inputs:
   * prefill, B=1, S=4096, 64 query / 8 key-value heads, head_dim 64: a
@@ -557,15 +557,159 @@ def run_long(args, name: str):
     return 0
 
 
+def run_chunk(args):
+    """One GPU: a step is a 4096-token chunk prefilled against a 12288-token
+    cached prefix (gptoss_attn_prefill_chunk), for a full-causal and a W=128
+    layer, each with its own cache. Prints one JSON line."""
+    import torch
+
+    import attention_gqa_b200 as gqa
+    from attention_gqa_b200 import build
+    build.build()
+    B, L, start, n = 1, 16384, 12288, 4096
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    gqa.init()
+    stream = torch.cuda.current_stream()
+    layers = []
+    for layer, window in ((0, 0), (1, 128)):
+        def draw(shape, tid):
+            g = torch.Generator(device=dev)
+            g.manual_seed(0x6A77 ^ (6 << 24) ^ (layer << 12) ^ tid)
+            return torch.randn(shape, generator=g, device=dev, dtype=torch.float32)
+        q = draw((B, L, NQ, D), 1).to(torch.bfloat16)
+        k = draw((B, L, NKV, D), 2).to(torch.bfloat16)
+        v = draw((B, L, NKV, D), 3).to(torch.bfloat16)
+        sinks = draw((NQ,), 4)
+        pos = torch.arange(L, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
+        kc = torch.empty(B, L, NKV, D, dtype=torch.bfloat16, device=dev)
+        vc = torch.empty_like(kc)
+        # the cached prefix, written once (untimed)
+        gqa.prefill_chunk(q[:, :start].contiguous(), k[:, :start].contiguous(),
+                          v[:, :start].contiguous(), sinks, pos[:, :start].contiguous(), kc, vc,
+                          0, window)
+        layers.append(dict(q=q, k=k, v=v, sinks=sinks, pos=pos, window=window, kc=kc, vc=vc,
+                           cq=q[:, start:].contiguous(), ck=k[:, start:].contiguous(),
+                           cv=v[:, start:].contiguous(), cp=pos[:, start:].contiguous(),
+                           out=torch.empty(B, n, NQ, D, dtype=torch.bfloat16, device=dev)))
+    gqa.check()
+    steps = max(1, min(args.steps, 20))
+
+    def step(ev=None):
+        for i, p in enumerate(layers):
+            if ev is not None:
+                ev[i].record(stream)
+            gqa.prefill_chunk(p["cq"], p["ck"], p["cv"], p["sinks"], p["cp"], p["kc"], p["vc"],
+                              start, p["window"], out=p["out"])
+        if ev is not None:
+            ev[len(layers)].record(stream)
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    gqa.check()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(layers) + 1)]
+              for _ in range(steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        for s_ in range(steps):
+            flush.fill_(s_ & 0xFF)
+            step(events[s_])
+        torch.cuda.synchronize()
+    gqa.check()
+    seg = np.array([[events[s_][i].elapsed_time(events[s_][i + 1]) for i in range(len(layers))]
+                    for s_ in range(steps)]).sum(axis=0) / steps
+    pairs = [n * start + n * (n + 1) // 2, 128 * n]      # visible pairs of the chunk's queries
+    flops = [4.0 * D * NQ * B * p for p in pairs]
+    step_ms = float(seg.sum())
+    value = sum(flops) / (step_ms * 1e-3) / 1e12
+    full_tf = flops[0] / (seg[0] * 1e-3) / 1e12
+    hbm, tf_burst, tf_sus, peak_src = load_peaks()
+    # e2e: the chunk's inputs from pinned host memory, its output back, per layer
+    p = layers[0]
+    host = [t.cpu().pin_memory() for t in (p["cq"], p["ck"], p["cv"], p["sinks"], p["cp"])]
+    dbuf = [torch.empty_like(t, device=dev) for t in host]
+    hout = torch.empty(p["out"].shape, dtype=torch.bfloat16).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for d_, h_ in zip(dbuf, host):
+        d_.copy_(h_, non_blocking=True)
+    gqa.prefill_chunk(dbuf[0], dbuf[1], dbuf[2], dbuf[3], dbuf[4], p["kc"], p["vc"], start, 0,
+                      out=p["out"])
+    hout.copy_(p["out"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_tf = flops[0] / (e0.elapsed_time(e1) * 1e-3) / 1e12
+    cpu_v, cpu_s, cpu_rows, cpu_flops = oracle_chunk_sample(layers[0], start, n)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: N(0,1) bf16 q/k/v and fp32 sinks drawn on the device (torch "
+                "generator seeded per layer), pos = token index",
+        "config": {"workload": "chunked prefill B=1: 4096 new tokens after 12288 cached ones "
+                               "(cache 16384), one full-causal layer + one W=128 layer",
+                   "l2": "flushed before every step (256 MB write)",
+                   "full_layer_ms": float(seg[0]), "full_layer_tflops": full_tf,
+                   "sliding_layer_ms": float(seg[1])},
+        "roofline": {"kernel": "chunked prefill (value copy + key rotation + prefill_kernel, "
+                               "full-causal layer)", "bound": "tensor", "achieved": full_tf,
+                     "peak": tf_burst, "unit": "TFLOP/s", "frac": full_tf / tf_burst,
+                     "peak_source": peak_src + " (burst)", "traffic": None,
+                     "launch_ms": float(seg[0])},
+        "cpu_baseline": {"value": cpu_v, "unit": "TFLOP/s", "cores": host_cores(),
+                         "kind": "oracle",
+                         "sample": "%d evenly spaced query rows (all 64 heads) of the full-causal "
+                                   "chunk, %.3g unmasked FLOPs, %.1f s"
+                                   % (cpu_rows, cpu_flops, cpu_s)},
+        "e2e": {"value": e2e_tf, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host),
+                "d2h_bytes_per_step": hout.numel() * hout.element_size(),
+                "what": "the full-causal chunk with its inputs from pinned host memory"},
+        "gpu_launches": steps * 2 * len(layers),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def oracle_chunk_sample(p, start: int, n: int, budget_s: float = 6.0):
+    """The fp64 oracle on evenly spaced query rows of a chunk (keys: the whole
+    cached prefix plus the chunk); returns (TFLOP/s, s, rows, FLOPs)."""
+    import oracle
+    oracle._load()
+    kh = p["k"].double().cpu().numpy()
+    vh = p["v"].double().cpu().numpy()
+    sh = p["sinks"].double().cpu().numpy()
+    ph = p["pos"].cpu().numpy()
+    m = 8
+    while True:
+        toks = start + np.linspace(0, n - 1, m).astype(np.int64)
+        rows = [(0, int(t)) for t in toks]
+        q_rows = np.stack([p["q"][0, t].double().cpu().numpy() for _, t in rows])
+        t0 = time.perf_counter()
+        oracle.prefill_rows(q_rows, kh, vh, sh, ph, p["window"], rows)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s / 3 or m >= 4096:
+            break
+        m *= 4
+    flops = sum(4.0 * D * NQ * (t + 1) for t in toks)
+    return flops / dt / 1e12, dt, m, flops
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["step"] + sorted(LONG_WORKLOADS), default="step",
+    ap.add_argument("--workload", choices=["step", "chunk16k"] + sorted(LONG_WORKLOADS),
+                    default="step",
                     help="step: the default prefill + decode step; tiny256 / batch16k / "
-                         "seq128k: other prefill workloads (one GPU, at most 20 timed steps)")
+                         "seq128k: other prefill workloads; chunk16k: chunked prefill against "
+                         "a cache (one GPU, at most 20 timed steps)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -577,6 +721,8 @@ def main():
         if world > 1:
             print("--workload %s runs on one GPU" % args.workload, file=sys.stderr)
             return 2
+        if args.workload == "chunk16k":
+            return run_chunk(args)
         return run_long(args, args.workload)
     return run_ours(args, rank, world)
 
