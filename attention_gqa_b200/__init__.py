@@ -9,6 +9,10 @@ device is missing, calls raise.
 Shapes (bf16 unless noted):
     prefill: q [B, S, 64, 64], k/v [B, S, 8, 64], sinks fp32 [64],
              pos int32 [B, S]  ->  out [B, S, 64, 64]
+    prefill_chunk: q [B, n, 64, 64], k/v [B, n, 8, 64], pos int32 [B, n],
+             kcache/vcache [B, L, 8, 64] holding `start` cached tokens
+             -> out [B, n, 64, 64]; the chunk's rotated keys and values are
+             written to rows [start, start+n) of the caches
     decode:  q [B, 64, 64] (un-rotated), kcache/vcache [B, L, 8, 64]
              (keys rotated), sinks fp32 [64], lengths int32 [B] -> out [B, 64, 64]
 ``window <= 0`` is full causal; ``window = W > 0`` the W-key sliding window.
