@@ -1,7 +1,7 @@
 """Throughput of the gpt-oss attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload step|tiny256|batch16k|seq128k|chunk16k]
+                    [--workload step|tiny256|batch16k|seq128k|layers36|chunk16k]
 
 One step is one pass of the whole path over one batch of synthetic inputs:
   * prefill, B=1, S=4096, 64 query / 8 key-value heads, head_dim 64: a
@@ -404,6 +404,10 @@ LONG_WORKLOADS = {
                  "alternating, each with its own inputs"),
     "seq128k": (5, 1, 131072, [(0, 0), (1, 128)],
                 "prefill B=1 S=131072 64q/8kv d64, one full-causal layer + one W=128 layer"),
+    # the 36-layer stack of the larger model: W=128 and full-causal layers alternating
+    "layers36": (7, 1, 4096, [(i, 128 if i % 2 == 0 else 0) for i in range(36)],
+                 "prefill B=1 S=4096 64q/8kv d64 through 36 layers, 18 W=128 + 18 full-causal "
+                 "alternating, each with its own inputs"),
 }
 
 
@@ -708,8 +712,8 @@ def main():
     ap.add_argument("--workload", choices=["step", "chunk16k"] + sorted(LONG_WORKLOADS),
                     default="step",
                     help="step: the default prefill + decode step; tiny256 / batch16k / "
-                         "seq128k: other prefill workloads; chunk16k: chunked prefill against "
-                         "a cache (one GPU, at most 20 timed steps)")
+                         "seq128k / layers36: other prefill workloads; chunk16k: chunked "
+                         "prefill against a cache (one GPU, at most 20 timed steps)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
