@@ -291,10 +291,32 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[e] += f * mw_base[hh * kHeadDim + d0 + e];
     }
-    const size_t row = (static_cast<size_t>(b) * kNumHeads + g * kGroup + hh) * a.nsplit + split;
-    *reinterpret_cast<float4*>(a.part_o + row * kHeadDim + d0) =
-        make_float4(acc[0], acc[1], acc[2], acc[3]);
-    if ((t & 15) == 0) a.part_ml[row] = make_float2(M, lsum);
+    const size_t head = static_cast<size_t>(b) * kNumHeads + g * kGroup + hh;
+    if (a.nsplit == 1) {
+      // one split covers the whole visible range: add the sink and normalise
+      // here (the combine step below, with a single split)
+      const float sink = __ldg(a.sinks + g * kGroup + hh);
+      const bool sink_off = isinf(sink) && sink < 0.f;
+      const float ms = sink_off ? -INFINITY : sink * kLog2e;
+      const float Mf = fmaxf(ms, M);
+      float den = 0.f, f = 0.f;
+      if (Mf != -INFINITY) {
+        den = sink_off ? 0.f : ex2_approx(ms - Mf);
+        if (M != -INFINITY) {
+          f = ex2_approx(M - Mf);
+          den += f * lsum;
+        }
+      }
+      const float scale = den > 0.f ? f / den : 0.f;
+      *reinterpret_cast<uint2*>(a.out + head * kHeadDim + d0) =
+          make_uint2(pack_bf16x2(acc[0] * scale, acc[1] * scale),
+                     pack_bf16x2(acc[2] * scale, acc[3] * scale));
+    } else {
+      const size_t row = head * a.nsplit + split;
+      *reinterpret_cast<float4*>(a.part_o + row * kHeadDim + d0) =
+          make_float4(acc[0], acc[1], acc[2], acc[3]);
+      if ((t & 15) == 0) a.part_ml[row] = make_float2(M, lsum);
+    }
   }
 }
 
@@ -340,6 +362,9 @@ void decode_plan(int batch, int max_len, int window, int* nsplit, int* chunk) {
   int ns = target_ctas / (batch * kNumKvHeads);
   const int max_ns = (n_plan + kKeys - 1) / kKeys;
   if (ns > max_ns) ns = max_ns;
+  // short visible ranges (sliding layers) take one split: each CTA then
+  // finishes its heads itself and the combine launch is skipped
+  if (n_plan <= 256) ns = 1;
   if (ns < 1) ns = 1;
   int ch = (n_plan + ns - 1) / ns;
   ch = (ch + kKeys - 1) / kKeys * kKeys;
@@ -362,6 +387,7 @@ cudaError_t launch_decode(const DecodeMaps& maps, const DecodeArgs& a, cudaStrea
   decode_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (a.nsplit == 1) return cudaSuccess;  // the split kernel wrote the output
   // programmatic dependent launch: the combine grid's launch overlaps the
   // split kernel's tail; its threads wait for the partials (griddep_wait).
   const int warps = a.batch * kNumHeads;
