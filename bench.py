@@ -381,8 +381,11 @@ def run_ours(args, rank: int, world: int):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "what": "prefill layers via host buffers"},
-            # per step: key rotation + attention per prefill layer, split-KV + combine per decode
-            "gpu_launches": args.steps * (2 * len(PREFILL_LAYERS) + 2 * len(DECODE_LAYERS)),
+            # per step: key rotation + attention per prefill layer; per decode layer the
+            # split kernel, plus the combine kernel unless one split covers the range
+            "gpu_launches": args.steps * (2 * len(PREFILL_LAYERS) + sum(
+                1 if (min(w, DECODE_L) if w > 0 else DECODE_L) <= 256 else 2
+                for _, w in DECODE_LAYERS)),
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
