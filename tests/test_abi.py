@@ -105,6 +105,12 @@ def test_workspace_query(lib):
     assert full >= slid > 0
     # per (batch, head, split): 64 fp32 partial outputs + (max, sum)
     assert full % (64 * 64 * (64 * 4 + 8)) == 0
+    # full-length layers split the keys over several CTAs (here 3 splits for 512
+    # (sequence, kv head) pairs); short visible ranges (<= 256 keys) take one split
+    assert full == 64 * 64 * 3 * (64 * 4 + 8)
+    assert slid == 64 * 64 * 1 * (64 * 4 + 8)
+    assert lib.gptoss_attn_decode_workspace_bytes(2, 256, 0) == 2 * 64 * (64 * 4 + 8)
+    assert lib.gptoss_attn_decode_workspace_bytes(2, 257, 0) > 2 * 64 * (64 * 4 + 8)
 
 
 def test_python_binding_refuses_without_device():
