@@ -632,14 +632,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Narrow-band kernel for sliding windows 0 < W <= 128 (the model's W = 128).
 //
 // Work item: batch b, kv head g, 16 query tokens = one M=128 tile. Query i
-// sees keys (i-W, i], so the whole item needs only the 144 keys
-// [q0-128, q0+16): one K/V span per item (TMA zero-fills rows before 0),
-// S = Q K^T with N = 144 and a single-tile softmax (no online rescaling).
-// Keys arrive already rotated; the RoPE warps rotate the item's Q rows.
-// Consecutive items alternate between the two softmax warpgroups so the
-// tensor core works on one item while the other's softmax runs. Each item's
-// Q, K and V share one ring stage; outputs go through a 4-slot staging ring
-// so the store of an item overlaps the next items' epilogues.
+// (key index q_start+i) sees keys (i-W, i], so the whole item needs only the
+// 144 keys [q0-128, q0+16): one K/V span per item (TMA zero-fills rows before
+// 0 and past the last key), S = Q K^T with N = 144 and a single-tile softmax
+// (no online rescaling). Keys arrive already rotated; the RoPE warps rotate
+// the item's Q rows. Consecutive items alternate between the two softmax
+// warpgroups so the tensor core works on one item while the other's softmax
+// runs; the single issuer issues an item's Q K^T and the previous item's P V
+// in whichever order their inputs land. Each item's Q, K, V and table rows
+// share one ring stage; outputs go through a 3-slot staging ring so the store
+// of an item overlaps the next items' epilogues.
 namespace band {
 
 constexpr int kTokens = 16;
