@@ -35,7 +35,12 @@
 // so Q K^T of tile j+1 overlaps the softmax of tile j and P.V of tile j
 // overlaps the softmax of tile j+1.
 // The running max starts at sigma*log2(e) with l = 1; O is rescaled only when
-// the max grows by more than 2^8 (exact: O and l share the reference).
+// the max grows by more than 2^8 (exact: O and l share the reference). The two
+// softmax warpgroups take turns on their exp loops (a warpgroup hands over 5/8
+// of the way through its loop), which keeps their tiles staggered against the
+// tensor core. Query token i of a call sits at key index q_start+i (q_start > 0
+// when a chunk is prefilled against a cache): masks and tile ranges use key
+// indices, Q rows, positions and outputs use i.
 #include <cmath>
 
 #include "internal.h"
