@@ -295,20 +295,49 @@ def decode_noalloc(q, kcache, vcache, sinks, lengths, window: int = 0, out=None,
     """decode() for callers that cannot allocate device memory: the split
     partials live in the library's fixed device array (GPTOSS_ATTN_NOALLOC_
     SCRATCH_BYTES) instead of a workspace. Device tensors only; pass `out` to
-    allocate nothing here either. Calls whose kernels overlap in time race."""
+    allocate nothing here either. Calls whose kernels overlap in time race.
+
+    Every argument's dtype, shape and contiguity is checked before the library
+    is touched, since the kernels derive their bounds from q and kcache."""
+    for name, t, dt in (("q", q, torch.bfloat16), ("kcache", kcache, torch.bfloat16),
+                        ("vcache", vcache, torch.bfloat16), ("sinks", sinks, torch.float32),
+                        ("lengths", lengths, torch.int32)):
+        if t.dtype != dt:
+            raise TypeError("%s must be %s, got %s" % (name, dt, t.dtype))
+        if not t.is_contiguous():
+            raise ValueError("%s must be contiguous" % name)
+    if q.dim() != 3 or tuple(q.shape[1:]) != (NUM_HEADS, HEAD_DIM):
+        raise ValueError("q must be [B, 64, 64], got %s" % (tuple(q.shape),))
+    B = q.shape[0]
+    if kcache.dim() != 4 or kcache.shape[0] != B or \
+            tuple(kcache.shape[2:]) != (NUM_KV_HEADS, HEAD_DIM):
+        raise ValueError("kcache must be [B, L, 8, 64] with B = %d, got %s"
+                         % (B, tuple(kcache.shape)))
+    if tuple(vcache.shape) != tuple(kcache.shape):
+        raise ValueError("vcache must match kcache %s, got %s"
+                         % (tuple(kcache.shape), tuple(vcache.shape)))
+    if tuple(sinks.shape) != (NUM_HEADS,):
+        raise ValueError("sinks must be [64], got %s" % (tuple(sinks.shape),))
+    if tuple(lengths.shape) != (B,):
+        raise ValueError("lengths must be [B] with B = %d, got %s" % (B, tuple(lengths.shape)))
+    if out is not None:
+        if out.dtype != torch.bfloat16 or not out.is_contiguous() or \
+                tuple(out.shape) != (B, NUM_HEADS, HEAD_DIM):
+            raise ValueError("out must be a contiguous bf16 [B, 64, 64] tensor, got %s %s"
+                             % (out.dtype, tuple(out.shape)))
+    device = q.device
+    if device.type != "cuda":
+        raise ValueError("decode_noalloc takes device tensors")
+    for name, t in (("kcache", kcache), ("vcache", vcache), ("sinks", sinks),
+                    ("lengths", lengths)) + ((("out", out),) if out is not None else ()):
+        if t.device != device:
+            raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
     lib = _load()
     fn = lib.gptoss_attn_decode_noalloc
     vp, i32 = ctypes.c_void_p, ctypes.c_int
     fn.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, vp]
     fn.restype = i32
-    device = q.device
-    if device.type != "cuda":
-        raise ValueError("decode_noalloc takes device tensors")
-    for name, t, dt in (("q", q, torch.bfloat16), ("kcache", kcache, torch.bfloat16),
-                        ("vcache", vcache, torch.bfloat16), ("sinks", sinks, torch.float32),
-                        ("lengths", lengths, torch.int32)):
-        _dev(t, dt, name, device)
-    B, L = q.shape[0], kcache.shape[1]
+    L = kcache.shape[1]
     if out is None:
         out = torch.empty((B, NUM_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=device)
     st = fn(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), sinks.data_ptr(),

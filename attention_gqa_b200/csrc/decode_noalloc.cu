@@ -1,13 +1,12 @@
 // Allocation-free decode entry point.
 //
-// Some callers cannot allocate device memory when they run decode: code that
-// records a CUDA graph (cudaMalloc is not allowed while a stream is being
-// captured), serving engines that hand all device memory to their own pool
-// up front and forbid later allocations, and latency-bound loops that cannot
-// afford the implicit synchronization of an allocation. For them this entry
-// point runs the same split-KV decode as gptoss_attn_decode(), but its scratch
-// (the per-split partial results and an error word) lives in a fixed array
-// that is part of the library's device image, so the call allocates nothing.
+// Some callers cannot allocate device memory when they run decode: serving
+// engines that hand all device memory to their own pool up front and forbid
+// later allocations, and latency-bound loops that cannot afford the implicit
+// synchronization of an allocation. For them this entry point runs the same
+// split-KV decode as gptoss_attn_decode(), but its scratch (the per-split
+// partial results and an error word) lives in a fixed array that is part of
+// the library's device image, so the call allocates nothing.
 //
 // The array is GPTOSS_ATTN_NOALLOC_SCRATCH_BYTES bytes on every GPU that loads
 // the library, held until the process exits. Every call shares it, so calls
@@ -37,7 +36,9 @@ std::mutex g_mutex;
 unsigned char* g_scratch_addr[kMaxDevices];  // device address of g_scratch, per device
 
 // Looks up the device address of the scratch array for `dev`, which must be
-// the current device. Done once per device; no allocation.
+// the current device. Done once per device ordinal and cached for the life of
+// the process (the address belongs to the device's primary context); no
+// allocation.
 int scratch_address(int dev, unsigned char** addr) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!g_scratch_addr[dev]) {

@@ -180,10 +180,9 @@ int gptoss_attn_decode(const void* q, const void* kcache, const void* vcache, co
 /*
  * Allocation-free decode. The gpt-oss pages have no counterpart: this entry
  * point exists for callers that cannot allocate device memory while they
- * decode, such as code recording a CUDA graph (allocation is not allowed
- * during stream capture), serving engines that give all device memory to
- * their own pool up front, and latency-bound loops that cannot pay for an
- * allocation's synchronization.
+ * decode, such as serving engines that give all device memory to their own
+ * pool up front and forbid later allocations, or latency-bound loops that
+ * cannot pay for the synchronization an allocation implies.
  *
  * Same operation and arguments as gptoss_attn_decode() without the
  * workspace: the split partials live in a fixed array of
@@ -196,11 +195,16 @@ int gptoss_attn_decode(const void* q, const void* kcache, const void* vcache, co
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture.
+ * The looked-up address is cached per device ordinal for the life of the
+ * process, which assumes the device's primary context throughout (no
+ * cudaDeviceReset, no other driver context current during these calls).
  * Every call shares the array, and a call clears only its error word before
  * launching, so calls whose kernels overlap in time on the GPU race: issue
  * them on one stream or otherwise serialize them. Device-side conditions of
  * this path (a length outside [0, max_len], which is clamped; a pipeline
- * timeout) are not reported by gptoss_attn_check().
+ * timeout) are not reported by gptoss_attn_check(), and this path keeps
+ * running while the device error word of the other entry points holds a
+ * timeout.
  */
 #define GPTOSS_ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
 

@@ -148,3 +148,43 @@ def test_prefill_chunk_argument_errors(lib):
     assert call(b=0) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
     assert call(vc=136) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
     assert call(p=82) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
+
+
+def test_decode_noalloc_binding_checks_shapes_before_the_library(monkeypatch):
+    """Each mis-shaped argument of decode_noalloc() raises before any library
+    call: the kernels take their bounds from q and kcache, so a wrong shape
+    that reached them would read or write out of bounds."""
+    import torch
+
+    def no_library():
+        raise AssertionError("the library was called")
+    monkeypatch.setattr(gqa, "_load", no_library)
+    B, L = 3, 40
+    good = dict(q=torch.zeros(B, 64, 64, dtype=torch.bfloat16),
+                kcache=torch.zeros(B, L, 8, 64, dtype=torch.bfloat16),
+                vcache=torch.zeros(B, L, 8, 64, dtype=torch.bfloat16),
+                sinks=torch.zeros(64, dtype=torch.float32),
+                lengths=torch.zeros(B, dtype=torch.int32))
+    bad = [
+        ("q", torch.zeros(B, 64, 32, dtype=torch.bfloat16)),
+        ("q", torch.zeros(B, 8, 64, 64, dtype=torch.bfloat16)),
+        ("kcache", torch.zeros(B + 1, L, 8, 64, dtype=torch.bfloat16)),
+        ("kcache", torch.zeros(B, L, 64, 64, dtype=torch.bfloat16)),
+        ("vcache", torch.zeros(B, L + 1, 8, 64, dtype=torch.bfloat16)),
+        ("vcache", torch.zeros(B - 1, L, 8, 64, dtype=torch.bfloat16)),
+        ("sinks", torch.zeros(8, dtype=torch.float32)),
+        ("lengths", torch.zeros(B + 2, dtype=torch.int32)),
+        ("kcache", torch.zeros(B, 8, L, 64, dtype=torch.bfloat16).transpose(1, 2)),
+    ]
+    for name, t in bad:
+        args = dict(good, **{name: t})
+        with pytest.raises(ValueError):
+            gqa.decode_noalloc(args["q"], args["kcache"], args["vcache"], args["sinks"],
+                               args["lengths"], 0)
+    with pytest.raises(ValueError):
+        gqa.decode_noalloc(*good.values(), 0, out=torch.zeros(B, 64, 63, dtype=torch.bfloat16))
+    with pytest.raises(TypeError):
+        gqa.decode_noalloc(*list(good.values())[:4], torch.zeros(B, dtype=torch.int64), 0)
+    # well-formed host tensors pass the shape checks and are refused as not on a device
+    with pytest.raises(ValueError, match="device tensors"):
+        gqa.decode_noalloc(*good.values(), 0)

@@ -1,8 +1,9 @@
 """The allocation-free decode entry point.
 
 gptoss_attn_decode_noalloc() serves callers that cannot allocate device
-memory while they decode (CUDA graph capture, engines that own all device
-memory in a pool, latency-bound loops). Its split partials live in a fixed
+memory while they decode (engines that own all device memory in a pool of
+their own, latency-bound loops that cannot pay for an allocation's
+synchronization). Its split partials live in a fixed
 array in the library's device image instead of a caller workspace. These
 tests call it through the C ABI and check it against gptoss_attn_decode()
 on the same inputs, twice in a row (the fixed array is reused by every call).
