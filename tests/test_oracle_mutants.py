@@ -43,12 +43,29 @@ MUTANTS = [
      "return pow(ROPE_THETA, -1.0 * (double)k / (double)D);",
      [pins.test_rope_unit_vectors_closed_form]),
     ("kv head h % 8 instead of h / 8",
-     "int h = g * GROUP + hh;\n            oracle_rope(q_rows",
-     "int h = hh * NKV + g;\n            oracle_rope(q_rows",
+     "int h = g * GROUP + hh;\n            rotate(q_rows",
+     "int h = hh * NKV + g;\n            rotate(q_rows",
      [lambda: pins.test_no_sink_no_rotation_equals_sdpa(0)]),
     ("scores not scaled",
      "s[j - lo] = dot * scale;", "s[j - lo] = dot;",
      [lambda: pins.test_no_sink_no_rotation_equals_sdpa(0), pins.test_window_one_closed_form]),
+    ("YaRN blend weights swapped (interpolate the high frequencies)",
+     "f[k] = inv_freq(k) / factor * ramp + inv_freq(k) * (1.0 - ramp);",
+     "f[k] = inv_freq(k) / factor * (1.0 - ramp) + inv_freq(k) * ramp;",
+     [pins.test_yarn_bands_and_attention_factor]),
+    ("YaRN attention factor left out",
+     "const double mscale = factor <= 1.0 ? 1.0 : 0.1 * log(factor) + 1.0;",
+     "const double mscale = 1.0;",
+     [pins.test_yarn_bands_and_attention_factor,
+      pins.test_yarn_attention_scales_logits_by_mscale_squared]),
+    ("YaRN correction pairs swapped between the betas",
+     "double lo = yarn_pair_for_turns(beta_fast, original);",
+     "double lo = yarn_pair_for_turns(beta_slow * 2.0, original);",
+     [pins.test_yarn_ramp_is_linear_in_the_pair_index]),
+    ("YaRN frequency ramp over turns instead of pair index",
+     "double ramp = ((double)k - lo) / (hi - lo);",
+     "double ramp = (original * inv_freq(k) / TWO_PI - beta_fast) / (beta_slow - beta_fast);",
+     [pins.test_yarn_ramp_is_linear_in_the_pair_index]),
     ("causal bound excludes the query itself",
      "attend_row(qr, kr, vg, (int64_t)NKV * D, lo, i, sinks[h], s, out + (r * NQ + h) * D);",
      "attend_row(qr, kr, vg, (int64_t)NKV * D, lo, i - 1, sinks[h], s, out + (r * NQ + h) * D);",
@@ -73,7 +90,8 @@ def test_pins_catch_planted_mistake(name, orig, mutated, checks):
     real = oracle._load()
     with tempfile.TemporaryDirectory() as tmp:
         lib = ctypes.CDLL(_build_mutant(src.replace(orig, mutated), tmp))
-        for fn in ("oracle_rope_rows", "oracle_prefill", "oracle_prefill_rows", "oracle_decode"):
+        for fn in ("oracle_rope_rows", "oracle_rope_yarn", "oracle_prefill", "oracle_prefill_rows",
+                   "oracle_decode"):
             getattr(lib, fn).argtypes = getattr(real, fn).argtypes
         caught = []
         oracle._lib = lib

@@ -141,6 +141,98 @@ def test_rope_norm_and_composition():
     assert np.allclose(oracle.rope(oracle.rope(x, a), b), oracle.rope(x, a + b), atol=1e-9)
 
 
+def _yarn_turn_rate(k, p=0.75, **kw):
+    """Angle per unit position that YaRN gives pair k (from one small rotation)."""
+    e = np.zeros(D); e[k] = 1.0
+    y = oracle.rope_yarn(e, p, **kw)
+    return math.atan2(y[k + 32], y[k]) / p, math.hypot(y[k], y[k + 32])
+
+
+def test_yarn_factor_one_is_plain_rope():
+    """With scaling factor 1 the interpolated and original frequencies agree and
+    the attention factor is 1: YaRN reduces to the plain rotation."""
+    rng = np.random.default_rng(21)
+    for p in (0.0, 1.0, 4095.0, 131071.0):
+        x = rng.standard_normal(D)
+        assert np.allclose(oracle.rope_yarn(x, p, factor=1.0), oracle.rope(x, p), atol=1e-12)
+
+
+def test_yarn_bands_and_attention_factor():
+    """NTK-by-parts structure of YaRN with s = 32 over a 4096-token original context:
+    pairs whose wavelength fits more than beta_fast = 32 times into the original
+    context keep their frequency; pairs fitting less than beta_slow = 1 time are
+    interpolated (frequency / 32, the same as the plain rotation at position p / 32);
+    every rotated vector is scaled by 0.1 ln 32 + 1."""
+    mscale = 0.1 * math.log(32.0) + 1.0
+    turns = [4096.0 * 150000.0 ** (-2.0 * k / 64) / (2 * math.pi) for k in range(32)]
+    for k in range(32):
+        rate, norm = _yarn_turn_rate(k)
+        assert norm == pytest.approx(mscale, rel=1e-13)
+        plain = 150000.0 ** (-2.0 * k / 64)
+        if turns[k] > 32.0:
+            assert rate == pytest.approx(plain, rel=1e-12), k
+        elif turns[k] < 1.0:
+            assert rate == pytest.approx(plain / 32.0, rel=1e-12), k
+        else:
+            assert plain / 32.0 < rate < plain, k
+    assert [k for k in range(32) if 1.0 <= turns[k] <= 32.0] == list(range(9, 18))
+    rng = np.random.default_rng(22)
+    x = rng.standard_normal(D)
+    x[:18] = 0.0
+    x[32:50] = 0.0                            # only interpolated pairs 18..31
+    p = 77777.0
+    assert np.allclose(oracle.rope_yarn(x, p), mscale * oracle.rope(x, p / 32.0), atol=1e-9)
+    # the model's mode of the row-rotation entry is this same rotation
+    assert np.allclose(oracle.rope(x[None], np.array([p]), rope="yarn")[0], oracle.rope_yarn(x, p),
+                       atol=1e-15)
+
+
+def test_yarn_ramp_is_linear_in_the_pair_index():
+    """Between the two correction pairs the blend weight of the interpolated
+    frequency rises linearly with the pair index (the transformers yarn ramp),
+    not linearly with the number of turns: the weights of pairs 9..17 have zero
+    second differences and reach 0 and 1 where the pair index where the
+    wavelength fits 32 resp. 1 times into 4096 tokens."""
+    w = []
+    for k in range(32):
+        rate, _ = _yarn_turn_rate(k)
+        plain = 150000.0 ** (-2.0 * k / 64)
+        w.append((plain - rate) / (plain - plain / 32.0))   # 0: original, 1: interpolated
+    w = np.array(w)
+    assert np.all(w[:9] == pytest.approx(0.0, abs=1e-12))
+    assert np.all(w[18:] == pytest.approx(1.0, abs=1e-12))
+    assert np.allclose(np.diff(w[9:18], 2), 0.0, atol=1e-10)
+    # the straight line through the ramp hits 0 and 1 at the correction pairs,
+    # where 4096 * theta^(-2k/64) / (2 pi) equals 32 and 1
+    slope = w[10] - w[9]
+    k0 = 9 - w[9] / slope
+    k1 = k0 + 1.0 / slope
+    assert 4096.0 * 150000.0 ** (-2.0 * k0 / 64) / (2 * math.pi) == pytest.approx(32.0, rel=1e-9)
+    assert 4096.0 * 150000.0 ** (-2.0 * k1 / 64) / (2 * math.pi) == pytest.approx(1.0, rel=1e-9)
+
+
+def test_yarn_attention_scales_logits_by_mscale_squared():
+    """With YaRN both q and k carry the attention factor, so at positions 0 the
+    output equals plain attention with q scaled by (0.1 ln 32 + 1)^2."""
+    B, S = 1, 12
+    rng = np.random.default_rng(23)
+    q = rng.standard_normal((B, S, NQ, D))
+    k = rng.standard_normal((B, S, NKV, D))
+    v = rng.standard_normal((B, S, NKV, D))
+    sinks = rng.standard_normal(NQ)
+    pos = np.zeros((B, S))
+    m2 = (0.1 * math.log(32.0) + 1.0) ** 2
+    got = oracle.prefill(q, k, v, sinks, pos, 5, rope="yarn")
+    assert np.allclose(got, oracle.prefill(q * m2, k, v, sinks, pos, 5), atol=1e-12)
+    dec = oracle.decode(q[:, -1], oracle.rope(k, np.zeros((B, S, NKV)), rope="yarn"), v, sinks,
+                        [S], 5, rope="yarn")
+    pos2 = np.broadcast_to(np.arange(S, dtype=np.float64), (B, S)).copy()
+    full = oracle.prefill(q, k, v, sinks, pos2, 5, rope="yarn")
+    kr = oracle.rope(k, pos2[:, :, None] * np.ones((1, 1, NKV)), rope="yarn")
+    dec = oracle.decode(q[:, -1], kr, v, sinks, [S], 5, rope="yarn")
+    assert np.allclose(dec, full[:, -1], atol=1e-12)
+
+
 def test_relative_position_invariance():
     """Shifting every position by a constant leaves the output unchanged."""
     q, k, v, s, pos = _rand_inputs(100, 1, 40)
@@ -308,3 +400,24 @@ def test_decode_empty_cache_is_zero():
     q = np.ones((2, NQ, D)); kc = np.ones((2, 4, NKV, D)); vc = np.ones((2, 4, NKV, D))
     o = oracle.decode(q, kc, vc, np.zeros(NQ), np.array([0, 0]), 0)
     assert np.all(o == 0.0)
+
+
+def test_torch_evaluation_of_the_input_recipe_matches_numpy():
+    """synth.device evaluates the same seeded recipe with torch (used for the
+    large bench and full-size test inputs); on the CPU it gives the numpy
+    generator's values exactly, including slices drawn on their own."""
+    import torch
+    from synth import device as sdev
+    seed = synth.seed_for(5, 1, synth.TENSOR_V)
+    w = sdev.splitmix64(seed, 12345, 1000, "cpu").numpy().view(np.uint64)
+    assert np.array_equal(w, synth.splitmix64(seed, 12345, 1000))
+    host = synth.bf16_normal(seed, (5, 300, 64))
+    got = sdev.bf16_normal(seed, (5, 300, 64), "cpu").view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, host)
+    part = sdev.bf16_normal_range(seed, 2 * 4567, 3000, "cpu").view(torch.int16).numpy()
+    assert np.array_equal(part.view(np.uint16), host.reshape(-1)[2 * 4567:2 * 4567 + 3000])
+    assert np.array_equal(synth.bf16_normal_range(seed, 2 * 4567, 3000),
+                          host.reshape(-1)[2 * 4567:2 * 4567 + 3000])
+    sinks = synth.seed_for(5, 1, synth.TENSOR_SINKS)
+    assert np.array_equal(sdev.f32_normal(sinks, (64,), "cpu").numpy(),
+                          synth.f32_normal(sinks, (64,)))
