@@ -16,6 +16,9 @@ Shapes (bf16 unless noted):
     decode:  q [B, 64, 64] (un-rotated), kcache/vcache [B, L, 8, 64]
              (keys rotated), sinks fp32 [64], lengths int32 [B] -> out [B, 64, 64]
 ``window <= 0`` is full causal; ``window = W > 0`` the W-key sliding window.
+``rope="yarn"`` selects the library's YaRN rotation (factor 32 over a
+4096-token original context) in place of plain RoPE; a cache filled with one
+rotation must be read with the same one.
 """
 from __future__ import annotations
 
@@ -24,7 +27,8 @@ import os
 
 import torch
 
-__all__ = ["prefill", "decode", "decode_noalloc", "prefill_workspace_bytes",
+__all__ = ["prefill", "prefill_lse", "prefill_backward", "decode", "decode_noalloc",
+           "prefill_workspace_bytes",
            "decode_workspace_bytes", "prefill_chunk", "check", "debug_wait_timeout", "init", "rope_table",
            "library_path", "GptossAttnError", "NUM_HEADS", "NUM_KV_HEADS", "HEAD_DIM",
            "MAX_POSITION"]
@@ -82,6 +86,22 @@ def _load():
     lib.gptoss_attn_check.restype = i32
     lib.gptoss_attn_debug_wait_timeout.argtypes = [ctypes.c_uint, vp]
     lib.gptoss_attn_debug_wait_timeout.restype = i32
+    lib.gptoss_attn_init_yarn.restype = i32
+    lib.gptoss_attn_rope_table_yarn.argtypes = [ctypes.POINTER(vp)]
+    lib.gptoss_attn_rope_table_yarn.restype = i32
+    lib.gptoss_attn_prefill_yarn.argtypes = lib.gptoss_attn_prefill.argtypes
+    lib.gptoss_attn_prefill_yarn.restype = i32
+    lib.gptoss_attn_prefill_chunk_yarn.argtypes = lib.gptoss_attn_prefill_chunk.argtypes
+    lib.gptoss_attn_prefill_chunk_yarn.restype = i32
+    lib.gptoss_attn_decode_yarn.argtypes = lib.gptoss_attn_decode.argtypes
+    lib.gptoss_attn_decode_yarn.restype = i32
+    lib.gptoss_attn_prefill_lse.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, vp, sz, vp]
+    lib.gptoss_attn_prefill_lse.restype = i32
+    lib.gptoss_attn_prefill_backward_workspace_bytes.argtypes = [i32, i32]
+    lib.gptoss_attn_prefill_backward_workspace_bytes.restype = sz
+    lib.gptoss_attn_prefill_backward.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp,
+                                                 vp, i32, i32, vp, sz, vp]
+    lib.gptoss_attn_prefill_backward.restype = i32
     if lib.gptoss_attn_abi_version() != ABI_VERSION:
         raise ImportError("%s has ABI %d, expected %d" % (path, lib.gptoss_attn_abi_version(),
                                                           ABI_VERSION))
@@ -125,9 +145,21 @@ def _target_device(*ts):
     return torch.device("cuda", torch.cuda.current_device())
 
 
-def init() -> None:
+ROPES = ("plain", "yarn")
+
+
+def _rope(rope: str) -> bool:
+    if rope not in ROPES:
+        raise ValueError("rope must be one of %s, got %r" % (ROPES, rope))
+    return rope == "yarn"
+
+
+def init(rope: str = "plain") -> None:
     """Build the current device's rotary table (allocates; call before graph capture)."""
-    _raise(_load().gptoss_attn_init(), "gptoss_attn_init")
+    if _rope(rope):
+        _raise(_load().gptoss_attn_init_yarn(), "gptoss_attn_init_yarn")
+    else:
+        _raise(_load().gptoss_attn_init(), "gptoss_attn_init")
 
 
 class _DevicePtr:
@@ -138,10 +170,12 @@ class _DevicePtr:
                                          "data": (ptr, False), "version": 3}
 
 
-def rope_table() -> torch.Tensor:
+def rope_table(rope: str = "plain") -> torch.Tensor:
     """A copy of the device rotary table, fp32 [131072, 32, 2] of (cos, sin)."""
     p = ctypes.c_void_p()
-    _raise(_load().gptoss_attn_rope_table(ctypes.byref(p)), "gptoss_attn_rope_table")
+    lib = _load()
+    fn = lib.gptoss_attn_rope_table_yarn if _rope(rope) else lib.gptoss_attn_rope_table
+    _raise(fn(ctypes.byref(p)), "gptoss_attn_rope_table")
     view = torch.as_tensor(_DevicePtr(p.value, (MAX_POSITION, HEAD_DIM // 2, 2), "<f4"),
                            device="cuda")
     return view.clone()
@@ -152,7 +186,7 @@ def prefill_workspace_bytes(batch: int, seqlen: int) -> int:
 
 
 def prefill(q, k, v, sinks, pos, window: int = 0, out=None, workspace=None,
-            stream=None) -> torch.Tensor:
+            stream=None, rope: str = "plain") -> torch.Tensor:
     """Causal grouped-query attention with sinks over whole sequences.
 
     Host (CPU) tensors are copied to the current CUDA device first and the
@@ -168,7 +202,8 @@ def prefill(q, k, v, sinks, pos, window: int = 0, out=None, workspace=None,
                 res = prefill(q.to(device, non_blocking=True), k.to(device, non_blocking=True),
                               v.to(device, non_blocking=True),
                               sinks.to(device, non_blocking=True),
-                              pos.to(device, non_blocking=True), window, None, workspace, s)
+                              pos.to(device, non_blocking=True), window, None, workspace, s,
+                              rope)
                 if out is None:
                     out = torch.empty(res.shape, dtype=res.dtype, pin_memory=True)
                 out.copy_(res, non_blocking=True)
@@ -193,17 +228,93 @@ def prefill(q, k, v, sinks, pos, window: int = 0, out=None, workspace=None,
         (B, S, NUM_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=device)
     if workspace is None:
         workspace = torch.empty(prefill_workspace_bytes(B, S), dtype=torch.uint8, device=device)
-    st = lib.gptoss_attn_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), sinks.data_ptr(),
-                                 pos.data_ptr(), int(window), dev_out.data_ptr(), B, S,
-                                 workspace.data_ptr(),
-                                 workspace.numel() * workspace.element_size(),
-                                 _stream_handle(stream))
+    fn = lib.gptoss_attn_prefill_yarn if _rope(rope) else lib.gptoss_attn_prefill
+    st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), sinks.data_ptr(), pos.data_ptr(),
+            int(window), dev_out.data_ptr(), B, S, workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _raise(st, "gptoss_attn_prefill")
     return dev_out
 
 
+def _prefill_shapes(q, k, v, sinks, pos, device):
+    q = _dev(q, torch.bfloat16, "q", device)
+    k = _dev(k, torch.bfloat16, "k", device)
+    v = _dev(v, torch.bfloat16, "v", device)
+    sinks = _dev(sinks, torch.float32, "sinks", device)
+    pos = _dev(pos, torch.int32, "pos", device)
+    if q.dim() != 4 or q.shape[2:] != (NUM_HEADS, HEAD_DIM):
+        raise ValueError("q must be [B, S, 64, 64], got %s" % (tuple(q.shape),))
+    B, S = q.shape[0], q.shape[1]
+    for name, t in (("k", k), ("v", v)):
+        if tuple(t.shape) != (B, S, NUM_KV_HEADS, HEAD_DIM):
+            raise ValueError("%s must be [B, S, 8, 64], got %s" % (name, tuple(t.shape)))
+    if tuple(sinks.shape) != (NUM_HEADS,) or tuple(pos.shape) != (B, S):
+        raise ValueError("sinks must be [64] and pos [B, S]")
+    return B, S
+
+
+def prefill_lse(q, k, v, sinks, pos, window: int = 0, out=None, lse=None, workspace=None,
+                stream=None):
+    """prefill() that also returns the natural-log softmax normaliser of every
+    query row (sink included), fp32 [B, S, 64], for prefill_backward(). Device
+    tensors only."""
+    lib = _load()
+    device = _target_device(q, k, v)
+    B, S = _prefill_shapes(q, k, v, sinks, pos, device)
+    if out is None:
+        out = torch.empty((B, S, NUM_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=device)
+    _dev(out, torch.bfloat16, "out", device)
+    if lse is None:
+        lse = torch.empty((B, S, NUM_HEADS), dtype=torch.float32, device=device)
+    _dev(lse, torch.float32, "lse", device)
+    if tuple(out.shape) != (B, S, NUM_HEADS, HEAD_DIM) or tuple(lse.shape) != (B, S, NUM_HEADS):
+        raise ValueError("out must be [B, S, 64, 64] and lse [B, S, 64]")
+    if workspace is None:
+        workspace = torch.empty(prefill_workspace_bytes(B, S), dtype=torch.uint8, device=device)
+    st = lib.gptoss_attn_prefill_lse(q.data_ptr(), k.data_ptr(), v.data_ptr(), sinks.data_ptr(),
+                                     pos.data_ptr(), int(window), out.data_ptr(), lse.data_ptr(),
+                                     B, S, workspace.data_ptr(),
+                                     workspace.numel() * workspace.element_size(),
+                                     _stream_handle(stream))
+    _raise(st, "gptoss_attn_prefill_lse")
+    return out, lse
+
+
+def prefill_backward_workspace_bytes(batch: int, seqlen: int) -> int:
+    return int(_load().gptoss_attn_prefill_backward_workspace_bytes(batch, seqlen))
+
+
+def prefill_backward(q, k, v, sinks, pos, window, out, lse, dout, workspace=None, stream=None):
+    """Gradients (dq, dk, dv bf16; dsinks fp32 [64]) of sum(dout * out) for the
+    prefill with these inputs; out and lse come from prefill_lse(). Device
+    tensors only."""
+    lib = _load()
+    device = _target_device(q, k, v)
+    B, S = _prefill_shapes(q, k, v, sinks, pos, device)
+    for name, t, dt, shape in (("out", out, torch.bfloat16, (B, S, NUM_HEADS, HEAD_DIM)),
+                               ("lse", lse, torch.float32, (B, S, NUM_HEADS)),
+                               ("dout", dout, torch.bfloat16, (B, S, NUM_HEADS, HEAD_DIM))):
+        _dev(t, dt, name, device)
+        if tuple(t.shape) != shape:
+            raise ValueError("%s must be %s, got %s" % (name, shape, tuple(t.shape)))
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    dsinks = torch.empty(NUM_HEADS, dtype=torch.float32, device=device)
+    if workspace is None:
+        workspace = torch.empty(prefill_backward_workspace_bytes(B, S), dtype=torch.uint8,
+                                device=device)
+    st = lib.gptoss_attn_prefill_backward(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), sinks.data_ptr(), pos.data_ptr(), int(window),
+        out.data_ptr(), lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+        dv.data_ptr(), dsinks.data_ptr(), B, S, workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _raise(st, "gptoss_attn_prefill_backward")
+    return dq, dk, dv, dsinks
+
+
 def prefill_chunk(q, k, v, sinks, pos, kcache, vcache, start: int, window: int = 0, out=None,
-                  stream=None) -> torch.Tensor:
+                  stream=None, rope: str = "plain") -> torch.Tensor:
     """Prefill of the next n = q.shape[1] tokens after `start` cached ones: writes
     their rotated keys and values into rows [start, start+n) of kcache / vcache
     ([B, max_len, 8, 64], device) and returns the chunk's attention output."""
@@ -231,10 +342,10 @@ def prefill_chunk(q, k, v, sinks, pos, kcache, vcache, start: int, window: int =
         raise ValueError("sinks must be [64] and pos [B, n]")
     dev_out = out if out is not None else torch.empty((B, n, NUM_HEADS, HEAD_DIM),
                                                       dtype=torch.bfloat16, device=device)
-    st = lib.gptoss_attn_prefill_chunk(q.data_ptr(), k.data_ptr(), v.data_ptr(), sinks.data_ptr(),
-                                       pos.data_ptr(), int(window), dev_out.data_ptr(),
-                                       kcache.data_ptr(), vcache.data_ptr(), B, int(start), n,
-                                       kcache.shape[1], _stream_handle(stream))
+    fn = lib.gptoss_attn_prefill_chunk_yarn if _rope(rope) else lib.gptoss_attn_prefill_chunk
+    st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), sinks.data_ptr(), pos.data_ptr(),
+            int(window), dev_out.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), B, int(start), n,
+            kcache.shape[1], _stream_handle(stream))
     _raise(st, "gptoss_attn_prefill_chunk")
     return dev_out
 
@@ -244,7 +355,7 @@ def decode_workspace_bytes(batch: int, max_len: int, window: int = 0) -> int:
 
 
 def decode(q, kcache, vcache, sinks, lengths, window: int = 0, out=None, workspace=None,
-           stream=None) -> torch.Tensor:
+           stream=None, rope: str = "plain") -> torch.Tensor:
     """One decode step against a rotated key cache; see the module docstring."""
     lib = _load()
     host = q.device.type != "cuda"
@@ -257,7 +368,8 @@ def decode(q, kcache, vcache, sinks, lengths, window: int = 0, out=None, workspa
                              kcache.to(device, non_blocking=True),
                              vcache.to(device, non_blocking=True),
                              sinks.to(device, non_blocking=True),
-                             lengths.to(device, non_blocking=True), window, None, workspace, s)
+                             lengths.to(device, non_blocking=True), window, None, workspace, s,
+                             rope)
                 if out is None:
                     out = torch.empty(res.shape, dtype=res.dtype, pin_memory=True)
                 out.copy_(res, non_blocking=True)
@@ -281,11 +393,10 @@ def decode(q, kcache, vcache, sinks, lengths, window: int = 0, out=None, workspa
         workspace = torch.empty(need, dtype=torch.uint8, device=device)
     dev_out = out if (out is not None and out.device.type == "cuda") else torch.empty(
         (B, NUM_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=device)
-    st = lib.gptoss_attn_decode(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
-                                sinks.data_ptr(), lengths.data_ptr(), int(window),
-                                dev_out.data_ptr(), B, L, workspace.data_ptr(),
-                                workspace.numel() * workspace.element_size(),
-                                _stream_handle(stream))
+    fn = lib.gptoss_attn_decode_yarn if _rope(rope) else lib.gptoss_attn_decode
+    st = fn(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), sinks.data_ptr(),
+            lengths.data_ptr(), int(window), dev_out.data_ptr(), B, L, workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _raise(st, "gptoss_attn_decode")
     return dev_out
 

@@ -14,10 +14,14 @@ using namespace gqa;
 constexpr int kMaxDevices = 64;
 
 struct DeviceState {
-  int* err = nullptr;       // 4-byte error word
-  float2* rope = nullptr;   // [kMaxPosition][32]
+  int* err = nullptr;         // 4-byte error word
+  float2* rope = nullptr;     // [kMaxPosition][32], plain RoPE
+  float2* yarn = nullptr;     // [kMaxPosition][32], YaRN (built on first use)
   int num_sms = 0;
 };
+
+// Which rotary table a call rotates with.
+enum class Rope { kNone, kPlain, kYarn };
 
 std::mutex g_mutex;
 DeviceState g_state[kMaxDevices];
@@ -32,9 +36,22 @@ int current_device(int* dev) {
   return GPTOSS_ATTN_OK;
 }
 
-// Allocates the error word (and, when asked, builds the rotary table) once
+// Builds one rotary table on the current device (legacy default stream, waited on).
+int build_table(float2** dst, bool yarn) {
+  float2* t = nullptr;
+  if (cudaMalloc(&t, sizeof(float2) * kMaxPosition * kRopePairs) != cudaSuccess)
+    return GPTOSS_ATTN_ERR_ALLOC;
+  if (launch_rope_table(t, yarn, nullptr) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(t);
+    return GPTOSS_ATTN_ERR_LAUNCH;
+  }
+  *dst = t;
+  return GPTOSS_ATTN_OK;
+}
+
+// Allocates the error word (and, when asked, builds a rotary table) once
 // per device. Runs on the legacy default stream and waits for completion.
-int ensure_state(int dev, bool need_rope) {
+int ensure_state(int dev, Rope need) {
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceState& st = g_state[dev];
   if (st.num_sms == 0 &&
@@ -49,17 +66,13 @@ int ensure_state(int dev, bool need_rope) {
     }
     st.err = e;
   }
-  if (need_rope && !st.rope) {
-    float2* t = nullptr;
-    if (cudaMalloc(&t, sizeof(float2) * kMaxPosition * kRopePairs) != cudaSuccess)
-      return GPTOSS_ATTN_ERR_ALLOC;
-    if (launch_rope_table(t, nullptr) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
-      cudaFree(t);
-      return GPTOSS_ATTN_ERR_LAUNCH;
-    }
-    st.rope = t;
-  }
+  if (need == Rope::kPlain && !st.rope) return build_table(&st.rope, false);
+  if (need == Rope::kYarn && !st.yarn) return build_table(&st.yarn, true);
   return GPTOSS_ATTN_OK;
+}
+
+const float2* table_of(int dev, Rope r) {
+  return r == Rope::kYarn ? g_state[dev].yarn : g_state[dev].rope;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -92,28 +105,41 @@ int gptoss_attn_init(void) {
   int dev = 0;
   int st = current_device(&dev);
   if (st != GPTOSS_ATTN_OK) return st;
-  return ensure_state(dev, true);
+  return ensure_state(dev, Rope::kPlain);
 }
 
-int gptoss_attn_rope_table(const void** table) {
+int gptoss_attn_init_yarn(void) {
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st != GPTOSS_ATTN_OK) return st;
+  return ensure_state(dev, Rope::kYarn);
+}
+
+static int rope_table_of(const void** table, Rope r) {
   if (!table) return GPTOSS_ATTN_ERR_NULL_PTR;
   int dev = 0;
   int st = current_device(&dev);
-  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, true);
+  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, r);
   if (st != GPTOSS_ATTN_OK) return st;
-  *table = g_state[dev].rope;
+  *table = table_of(dev, r);
   return GPTOSS_ATTN_OK;
 }
+
+int gptoss_attn_rope_table(const void** table) { return rope_table_of(table, Rope::kPlain); }
+
+int gptoss_attn_rope_table_yarn(const void** table) { return rope_table_of(table, Rope::kYarn); }
 
 size_t gptoss_attn_prefill_workspace_bytes(int batch, int seqlen) {
   if (batch < 1 || seqlen < 1 || seqlen > kMaxPosition || batch > 65535) return 0;
   return static_cast<size_t>(batch) * seqlen * kNumKvHeads * kHeadDim * 2;
 }
 
-int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float* sinks,
+static int prefill_impl(const void* q, const void* k, const void* v, const float* sinks,
                         const int32_t* pos, int window, void* out, int batch, int seqlen,
-                        void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream, Rope rope,
+                        float* lse) {
   if (!q || !k || !v || !sinks || !pos || !out || !workspace) return GPTOSS_ATTN_ERR_NULL_PTR;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GPTOSS_ATTN_ERR_BAD_ALIGN;
   if (batch < 1 || seqlen < 1 || seqlen > kMaxPosition || batch > 65535)
     return GPTOSS_ATTN_ERR_BAD_SHAPE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
@@ -124,7 +150,7 @@ int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float
     return GPTOSS_ATTN_ERR_SMALL_WORKSPACE;
   int dev = 0;
   int st = current_device(&dev);
-  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, true);
+  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, rope);
   if (st != GPTOSS_ATTN_OK) return st;
 
   PrefillMaps maps;
@@ -149,8 +175,9 @@ int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float
   PrefillArgs args;
   args.pos = pos;
   args.sinks = sinks;
-  args.rope = g_state[dev].rope;
+  args.rope = table_of(dev, rope);
   args.err = g_state[dev].err;
+  args.lse = lse;
   args.batch = batch;
   args.seqlen = seqlen;
   args.q_start = 0;
@@ -166,10 +193,10 @@ int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float
                                                            : GPTOSS_ATTN_ERR_LAUNCH;
 }
 
-int gptoss_attn_prefill_chunk(const void* q, const void* k, const void* v, const float* sinks,
+static int prefill_chunk_impl(const void* q, const void* k, const void* v, const float* sinks,
                               const int32_t* pos, int window, void* out, void* kcache,
                               void* vcache, int batch, int start, int n, int max_len,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, Rope rope) {
   if (!q || !k || !v || !sinks || !pos || !out || !kcache || !vcache)
     return GPTOSS_ATTN_ERR_NULL_PTR;
   if (batch < 1 || batch > 65535 || n < 1 || start < 0 || max_len > kMaxPosition ||
@@ -181,7 +208,7 @@ int gptoss_attn_prefill_chunk(const void* q, const void* k, const void* v, const
     return GPTOSS_ATTN_ERR_BAD_ALIGN;
   int dev = 0;
   int st = current_device(&dev);
-  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, true);
+  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, rope);
   if (st != GPTOSS_ATTN_OK) return st;
 
   const int keys = start + n;  // keys visible to the chunk: the cached prefix and the chunk
@@ -209,8 +236,9 @@ int gptoss_attn_prefill_chunk(const void* q, const void* k, const void* v, const
   PrefillArgs args;
   args.pos = pos;
   args.sinks = sinks;
-  args.rope = g_state[dev].rope;
+  args.rope = table_of(dev, rope);
   args.err = g_state[dev].err;
+  args.lse = nullptr;
   args.batch = batch;
   args.seqlen = n;
   args.q_start = start;
@@ -241,12 +269,14 @@ size_t gptoss_attn_decode_workspace_bytes(int batch, int max_len, int window) {
   return decode_workspace_bytes(batch, nsplit);
 }
 
-int gptoss_attn_decode(const void* q, const void* kcache, const void* vcache, const float* sinks,
+static int decode_impl(const void* q, const void* kcache, const void* vcache, const float* sinks,
                        const int32_t* len, int window, void* out, int batch, int max_len,
-                       void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream, Rope rope) {
   if (!q || !kcache || !vcache || !sinks || !len || !out || !workspace)
     return GPTOSS_ATTN_ERR_NULL_PTR;
   if (batch < 1 || max_len < 1 || batch > 65535) return GPTOSS_ATTN_ERR_BAD_SHAPE;
+  // the YaRN table covers positions below 131072
+  if (rope == Rope::kYarn && max_len > kMaxPosition) return GPTOSS_ATTN_ERR_BAD_SHAPE;
   if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out) ||
       !aligned16(workspace) || (reinterpret_cast<uintptr_t>(sinks) & 3u) ||
       (reinterpret_cast<uintptr_t>(len) & 3u))
@@ -257,7 +287,7 @@ int gptoss_attn_decode(const void* q, const void* kcache, const void* vcache, co
   if (workspace_bytes < need) return GPTOSS_ATTN_ERR_SMALL_WORKSPACE;
   int dev = 0;
   int st = current_device(&dev);
-  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, false);
+  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, rope == Rope::kYarn ? Rope::kYarn : Rope::kNone);
   if (st != GPTOSS_ATTN_OK) return st;
 
   DecodeMaps maps;
@@ -276,6 +306,7 @@ int gptoss_attn_decode(const void* q, const void* kcache, const void* vcache, co
   a.vcache = static_cast<const uint16_t*>(vcache);
   a.sinks = sinks;
   a.len = len;
+  a.rope = rope == Rope::kYarn ? table_of(dev, rope) : nullptr;
   a.out = static_cast<uint16_t*>(out);
   const size_t rows = static_cast<size_t>(batch) * kNumHeads * nsplit;
   a.part_o = static_cast<float*>(workspace);
@@ -289,11 +320,153 @@ int gptoss_attn_decode(const void* q, const void* kcache, const void* vcache, co
   return launch_decode(maps, a, stream) == cudaSuccess ? GPTOSS_ATTN_OK : GPTOSS_ATTN_ERR_LAUNCH;
 }
 
+int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float* sinks,
+                        const int32_t* pos, int window, void* out, int batch, int seqlen,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return prefill_impl(q, k, v, sinks, pos, window, out, batch, seqlen, workspace, workspace_bytes,
+                      stream, Rope::kPlain, nullptr);
+}
+
+int gptoss_attn_prefill_lse(const void* q, const void* k, const void* v, const float* sinks,
+                            const int32_t* pos, int window, void* out, float* lse, int batch,
+                            int seqlen, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream) {
+  if (!lse) return GPTOSS_ATTN_ERR_NULL_PTR;
+  return prefill_impl(q, k, v, sinks, pos, window, out, batch, seqlen, workspace, workspace_bytes,
+                      stream, Rope::kPlain, lse);
+}
+
+int gptoss_attn_prefill_yarn(const void* q, const void* k, const void* v, const float* sinks,
+                             const int32_t* pos, int window, void* out, int batch, int seqlen,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return prefill_impl(q, k, v, sinks, pos, window, out, batch, seqlen, workspace, workspace_bytes,
+                      stream, Rope::kYarn, nullptr);
+}
+
+int gptoss_attn_prefill_chunk(const void* q, const void* k, const void* v, const float* sinks,
+                              const int32_t* pos, int window, void* out, void* kcache,
+                              void* vcache, int batch, int start, int n, int max_len,
+                              cudaStream_t stream) {
+  return prefill_chunk_impl(q, k, v, sinks, pos, window, out, kcache, vcache, batch, start, n,
+                            max_len, stream, Rope::kPlain);
+}
+
+int gptoss_attn_prefill_chunk_yarn(const void* q, const void* k, const void* v,
+                                   const float* sinks, const int32_t* pos, int window, void* out,
+                                   void* kcache, void* vcache, int batch, int start, int n,
+                                   int max_len, cudaStream_t stream) {
+  return prefill_chunk_impl(q, k, v, sinks, pos, window, out, kcache, vcache, batch, start, n,
+                            max_len, stream, Rope::kYarn);
+}
+
+int gptoss_attn_decode(const void* q, const void* kcache, const void* vcache, const float* sinks,
+                       const int32_t* len, int window, void* out, int batch, int max_len,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return decode_impl(q, kcache, vcache, sinks, len, window, out, batch, max_len, workspace,
+                     workspace_bytes, stream, Rope::kPlain);
+}
+
+int gptoss_attn_decode_yarn(const void* q, const void* kcache, const void* vcache,
+                            const float* sinks, const int32_t* len, int window, void* out,
+                            int batch, int max_len, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream) {
+  return decode_impl(q, kcache, vcache, sinks, len, window, out, batch, max_len, workspace,
+                     workspace_bytes, stream, Rope::kYarn);
+}
+
+// Backward workspace: rotated q, rotated k, then lse2 and D in [b][g][t][8]
+// layout, each float array padded by one 128-row tile.
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+static void backward_layout(int batch, int seqlen, size_t off[5]) {
+  const size_t BS = static_cast<size_t>(batch) * seqlen;
+  off[0] = 0;
+  off[1] = align256(BS * kNumHeads * kHeadDim * 2);
+  off[2] = off[1] + align256(BS * kNumKvHeads * kHeadDim * 2);
+  off[3] = off[2] + align256((BS * kNumHeads + 128) * 4);
+  off[4] = off[3] + align256((BS * kNumHeads + 128) * 4);
+}
+
+size_t gptoss_attn_prefill_backward_workspace_bytes(int batch, int seqlen) {
+  if (batch < 1 || seqlen < 1 || seqlen > kMaxPosition || batch > 65535) return 0;
+  size_t off[5];
+  backward_layout(batch, seqlen, off);
+  return off[4];
+}
+
+int gptoss_attn_prefill_backward(const void* q, const void* k, const void* v, const float* sinks,
+                                 const int32_t* pos, int window, const void* out, const float* lse,
+                                 const void* dout, void* dq, void* dk, void* dv, float* dsinks,
+                                 int batch, int seqlen, void* workspace, size_t workspace_bytes,
+                                 cudaStream_t stream) {
+  if (!q || !k || !v || !sinks || !pos || !out || !lse || !dout || !dq || !dk || !dv ||
+      !dsinks || !workspace)
+    return GPTOSS_ATTN_ERR_NULL_PTR;
+  if (batch < 1 || seqlen < 1 || seqlen > kMaxPosition || batch > 65535)
+    return GPTOSS_ATTN_ERR_BAD_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(sinks) & 3u) || (reinterpret_cast<uintptr_t>(pos) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(dsinks) & 3u))
+    return GPTOSS_ATTN_ERR_BAD_ALIGN;
+  if (workspace_bytes < gptoss_attn_prefill_backward_workspace_bytes(batch, seqlen))
+    return GPTOSS_ATTN_ERR_SMALL_WORKSPACE;
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, Rope::kPlain);
+  if (st != GPTOSS_ATTN_OK) return st;
+
+  size_t off[5];
+  backward_layout(batch, seqlen, off);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  BackwardMaps maps;
+  const uint64_t S = static_cast<uint64_t>(seqlen), B = static_cast<uint64_t>(batch);
+  const uint64_t qdims[4] = {kHeadDim, kNumHeads, S, B};
+  const uint64_t qstr[3] = {kHeadDim * 2, kNumHeads * kHeadDim * 2, S * kNumHeads * kHeadDim * 2};
+  const uint32_t qbox[4] = {kHeadDim, kGroup, 16, 1};
+  const uint64_t kdims[4] = {kHeadDim, kNumKvHeads, S, B};
+  const uint64_t kstr[3] = {kHeadDim * 2, kNumKvHeads * kHeadDim * 2,
+                            S * kNumKvHeads * kHeadDim * 2};
+  const uint32_t kbox[4] = {kHeadDim, 1, 128, 1};
+  if (!make_tmap_bf16_4d(&maps.q, ws + off[0], qdims, qstr, qbox) ||
+      !make_tmap_bf16_4d(&maps.dout, dout, qdims, qstr, qbox) ||
+      !make_tmap_bf16_4d(&maps.k, ws + off[1], kdims, kstr, kbox) ||
+      !make_tmap_bf16_4d(&maps.v, v, kdims, kstr, kbox))
+    return GPTOSS_ATTN_ERR_TENSOR_MAP;
+
+  BackwardArgs a;
+  a.pos = pos;
+  a.sinks = sinks;
+  a.rope = table_of(dev, Rope::kPlain);
+  a.err = g_state[dev].err;
+  a.lse = lse;
+  a.out = static_cast<const uint16_t*>(out);
+  a.dout = static_cast<const uint16_t*>(dout);
+  a.lse2 = reinterpret_cast<float*>(ws + off[2]);
+  a.dd = reinterpret_cast<float*>(ws + off[3]);
+  a.dsinks = dsinks;
+  a.dq = static_cast<uint16_t*>(dq);
+  a.dk = static_cast<uint16_t*>(dk);
+  a.dv = static_cast<uint16_t*>(dv);
+  a.batch = batch;
+  a.seqlen = seqlen;
+  a.window = (window > 0 && window < seqlen) ? window : 0;
+  a.n_qt = backward_q_tiles(seqlen);
+  const int sms = g_state[dev].num_sms;
+  if (cudaMemsetAsync(dsinks, 0, kNumHeads * sizeof(float), stream) != cudaSuccess ||
+      launch_rope_rows(q, pos, a.rope, ws + off[0], batch, seqlen, seqlen, 0, kNumHeads, sms * 8,
+                       a.err, stream) != cudaSuccess ||
+      launch_rope_rows(k, pos, a.rope, ws + off[1], batch, seqlen, seqlen, 0, kNumKvHeads,
+                       sms * 8, a.err, stream) != cudaSuccess)
+    return GPTOSS_ATTN_ERR_LAUNCH;
+  return launch_backward(maps, a, sms, stream) == cudaSuccess ? GPTOSS_ATTN_OK
+                                                              : GPTOSS_ATTN_ERR_LAUNCH;
+}
+
 int gptoss_attn_debug_wait_timeout(unsigned timeout_us, cudaStream_t stream) {
   if (timeout_us == 0 || timeout_us > 2000000u) return GPTOSS_ATTN_ERR_BAD_SHAPE;
   int dev = 0;
   int st = current_device(&dev);
-  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, false);
+  if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, Rope::kNone);
   if (st != GPTOSS_ATTN_OK) return st;
   return launch_wait_timeout(g_state[dev].err, static_cast<uint64_t>(timeout_us) * 1000u,
                              stream) == cudaSuccess

@@ -1,0 +1,554 @@
+// Backward pass of the prefill attention for sm_100a: gradients of
+// L = sum(dO * out) with respect to q, k, v and the per-head sink logits
+// (the forward of the gpt-oss pages: inteligile "gpt-oss-120b" techniques map
+// rows "Grouped-query attention", "Partial RoPE", "Learnable attention sink",
+// "Sliding-window attention").
+//
+// With rotated q' = R(pos) q, k' = R(pos) k, scores s = q'.k'/8, the row
+// normaliser lse (sink included, from the forward) and p = exp(s - lse):
+//   D_i      = dO_i . out_i
+//   dS_ij    = p_ij (dO_i . v_j - D_i)
+//   dv_j     = sum_i p_ij dO_i            (the 8 heads of a group summed)
+//   dq'_i    = sum_j dS_ij k'_j / 8,  dk'_j = sum_i dS_ij q'_i / 8
+//   dsigma_h = -sum_i exp(sigma_h - lse_i) D_i
+//   dq = R(pos)^T dq',  dk = R(pos)^T dk'.
+//
+// Kernels, in stream order:
+//   rope_rows_kernel (twice): q' and k' into the workspace (bf16, as the
+//     forward rounds them for the tensor cores).
+//   bwd_prep_kernel: D and lse in log2 units per row, laid out [b][g][t][8]
+//     so a 16-token tile of one group is 128 consecutive floats; the sink
+//     gradient (block sums, one atomic per head and block).
+//   bwd_dq_kernel: one CTA per (b, g, 16 tokens) = an M=128 tile of 16 tokens
+//     x 8 heads; over its key tiles: S = Q'K'^T and dP = dO V^T (tcgen05, fp32
+//     in TMEM), dS by the elementwise warpgroup (bf16 back into S's columns),
+//     dQ += dS K' (A from TMEM). dQ stays in TMEM until the item's end, is
+//     rotated back and stored as bf16.
+//   bwd_dkv_kernel: one CTA per (b, g, 128 keys) = M=128 keys; over the
+//     query tiles that see them: S^T = K'Q'^T, dP^T = V dO^T, P^T and dS^T by
+//     the elementwise warpgroup, dV += P^T dO and dK += dS^T Q' (A from TMEM,
+//     summing over the 8 heads of the group because they are rows of the
+//     tile). No atomics on dq, dk or dv.
+// Roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
+// warps 4-7 the elementwise warpgroup (thread = TMEM lane); warps 2-3 idle.
+// Every pipeline wait is bounded like the forward kernels'.
+#include <cmath>
+
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace gqa {
+namespace {
+namespace bwd {
+
+constexpr int kThreads = 256;
+constexpr int kTok = 16;      // query tokens per 128-row tile
+constexpr int kKeys = 128;    // keys per tile
+constexpr int kStages = 2;
+constexpr uint32_t kTile = 128 * 128;  // 128 rows of 64 bf16
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kScaleLog2 = 0.125f * kLog2e;
+constexpr float kScale = 0.125f;
+// TMEM columns: S (or S^T) [0,128), dP (dP^T) [128,256), dQ or dV [256,320), dK [320,384).
+constexpr uint32_t kColS = 0, kColP = 128, kColA = 256, kColB = 320;
+
+// dq kernel shared memory
+constexpr uint32_t kQOffQ = 0, kQOffDO = kTile, kQOffK = 2 * kTile;
+constexpr uint32_t kQOffV = kQOffK + kStages * kTile;
+constexpr uint32_t kQOffBar = kQOffV + kStages * kTile;
+// dkv kernel shared memory
+constexpr uint32_t kKOffK = 0, kKOffV = kTile, kKOffQ = 2 * kTile;  // [stage]: Q', then dO
+constexpr uint32_t kKOffLD = kKOffQ + kStages * 2 * kTile;           // [stage]: lse2[128], D[128]
+constexpr uint32_t kKOffBar = kKOffLD + kStages * 1024;
+// one CTA per SM: the tensor memory allocation takes all 512 columns
+constexpr uint32_t kSmemBytes = 120 * 1024;
+static_assert(kQOffBar + 256 + 1024 <= kSmemBytes && kKOffBar + 256 + 1024 <= kSmemBytes, "smem");
+
+enum : int {
+  BAR_Q_FULL = 0,                        // [2] the query-side tile(s) of a stage
+  BAR_Q_EMPTY = BAR_Q_FULL + kStages,    // [2]
+  BAR_KV_FULL = BAR_Q_EMPTY + kStages,   // [2]
+  BAR_KV_EMPTY = BAR_KV_FULL + kStages,  // [2]
+  BAR_S_FULL = BAR_KV_EMPTY + kStages,   // S and dP written
+  BAR_E_DONE = BAR_S_FULL + 1,           // elementwise results in TMEM, S/dP read
+  BAR_ACC_FULL = BAR_E_DONE + 1,         // the item's accumulators complete
+  BAR_MMA_DONE = BAR_ACC_FULL + 1,
+  NUM_BARS = BAR_MMA_DONE + 1
+};
+
+struct Ctx {
+  uint32_t sbase, obar;
+  volatile int* abort_flag;
+  int* err;
+  __device__ uint32_t bar(int i) const { return sbase + obar + 8u * static_cast<uint32_t>(i); }
+  __device__ bool wait(int i, uint32_t parity) const {
+    return mbar_wait(bar(i), parity, abort_flag, err, kErrTimeout, kWaitTimeoutNs);
+  }
+  __device__ bool wait_warp(int i, uint32_t parity) const {
+    return mbar_wait_warp(bar(i), parity, abort_flag, err, kErrTimeout, kWaitTimeoutNs);
+  }
+};
+
+// Common prologue: barriers, abort flag (a timeout left in the error word
+// skips the work), tensor memory. Returns the TMEM base address.
+__device__ uint32_t setup(Ctx& ctx, uint8_t* smem, uint32_t obar, int* err) {
+  ctx.sbase = smem_u32(smem);
+  ctx.obar = obar;
+  ctx.abort_flag = reinterpret_cast<volatile int*>(smem + obar + NUM_BARS * 8 + 4);
+  ctx.err = err;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + obar + NUM_BARS * 8);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(ctx.bar(BAR_Q_FULL + s), 1);
+      mbar_init(ctx.bar(BAR_Q_EMPTY + s), 1);
+      mbar_init(ctx.bar(BAR_KV_FULL + s), 1);
+      mbar_init(ctx.bar(BAR_KV_EMPTY + s), 1);
+    }
+    mbar_init(ctx.bar(BAR_S_FULL), 1);
+    mbar_init(ctx.bar(BAR_E_DONE), 4);
+    mbar_init(ctx.bar(BAR_ACC_FULL), 1);
+    mbar_init(ctx.bar(BAR_MMA_DONE), 1);
+    *ctx.abort_flag = (*reinterpret_cast<volatile int*>(err) & kErrTimeout) ? 1 : 0;
+    fence_barrier_init();
+  }
+  if ((threadIdx.x >> 5) == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  return *tmem_slot;
+}
+
+__device__ void teardown(uint32_t tmem) {
+  tc_fence_before_sync();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// D = A B^T over head_dim 64 for two K-major 128-row tiles (4 MMAs, K = 16).
+__device__ __forceinline__ void mma_abt(uint32_t d_tmem, uint32_t a, uint32_t b) {
+  constexpr uint32_t idesc = idesc_bf16(128, 128, false);
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    mma_bf16_ss(d_tmem, sdesc_sw128(a + 32 * kk), sdesc_sw128(b + 32 * kk), idesc,
+                kk > 0 ? 1u : 0u);
+}
+
+// D (+)= A B with A bf16 [128 x 128] in TMEM and B a 128-row tile read
+// MN-major (rows = the contraction, 64 bf16 per row = the N columns).
+__device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint32_t b,
+                                           bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16(128, kHeadDim, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_bf16_ts(d_tmem, a_tmem + 8 * kk, sdesc_sw128(b + 2048 * kk), idesc,
+                (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// Rotates a 64-element gradient row back (R(p)^T) with the table row `cs`
+// (global memory) and stores it as bf16 at `dst` (128 bytes, 16-byte aligned).
+__device__ __forceinline__ void unrotate_store(const uint32_t (&lo)[32], const uint32_t (&hi)[32],
+                                               const float2* cs, uint16_t* dst) {
+  uint32_t w[32];
+#pragma unroll
+  for (int k = 0; k < 32; k += 2) {
+    const float4 t = __ldg(reinterpret_cast<const float4*>(cs + k));
+    const float y1a = __uint_as_float(lo[k]), y2a = __uint_as_float(hi[k]);
+    const float y1b = __uint_as_float(lo[k + 1]), y2b = __uint_as_float(hi[k + 1]);
+    w[k / 2] = pack_bf16x2(fmaf(y1a, t.x, y2a * t.y), fmaf(y1b, t.z, y2b * t.w));
+    w[16 + k / 2] = pack_bf16x2(fmaf(y2a, t.x, -y1a * t.y), fmaf(y2b, t.z, -y1b * t.w));
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+}
+
+__device__ __forceinline__ int clamp_pos(int p, int* err) {
+  if (p < 0 || p >= kMaxPosition) {
+    atomicOr(err, kErrPosition);
+    return p < 0 ? 0 : kMaxPosition - 1;
+  }
+  return p;
+}
+
+}  // namespace bwd
+
+// D and lse2 per row, and the sink gradient. Thread (token lane, head): 256
+// threads = 4 token lanes x 64 heads, grid-stride over tokens.
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BackwardArgs a) {
+  const int h = static_cast<int>(threadIdx.x & 63);
+  const int lane_t = static_cast<int>(threadIdx.x >> 6);
+  const int g = h / kGroup, hl = h % kGroup;
+  const float sig = __ldg(a.sinks + h);
+  const bool sink_on = !(isinf(sig) && sig < 0.f);
+  const int64_t ntok = static_cast<int64_t>(a.batch) * a.seqlen;
+  float acc = 0.f;
+  for (int64_t bt = static_cast<int64_t>(blockIdx.x) * 4 + lane_t; bt < ntok;
+       bt += static_cast<int64_t>(gridDim.x) * 4) {
+    const int64_t row = bt * kNumHeads + h;
+    const uint4* po = reinterpret_cast<const uint4*>(a.out + row * kHeadDim);
+    const uint4* pd = reinterpret_cast<const uint4*>(a.dout + row * kHeadDim);
+    float d = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint4 o = __ldg(po + i), g4 = __ldg(pd + i);
+      const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        d = fmaf(bf16lo_to_f32(ow[e]), bf16lo_to_f32(gw[e]),
+                 fmaf(bf16hi_to_f32(ow[e]), bf16hi_to_f32(gw[e]), d));
+    }
+    const float lse2 = __ldg(a.lse + row) * bwd::kLog2e;
+    const int64_t b = bt / a.seqlen, t = bt % a.seqlen;
+    const int64_t w = ((b * kNumKvHeads + g) * a.seqlen + t) * kGroup + hl;
+    a.lse2[w] = lse2;
+    a.dd[w] = d;
+    if (sink_on) acc -= ex2_approx(sig * bwd::kLog2e - lse2) * d;
+  }
+  __shared__ float red[4][64];
+  red[lane_t][h] = acc;
+  __syncthreads();
+  if (lane_t == 0) atomicAdd(a.dsinks + h, red[0][h] + red[1][h] + red[2][h] + red[3][h]);
+}
+
+// dQ for one (b, g, 16-token) tile per CTA.
+__global__ void __launch_bounds__(bwd::kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ BackwardMaps maps, const BackwardArgs a) {
+  using namespace bwd;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  Ctx ctx;
+  const uint32_t tmem = setup(ctx, smem, kQOffBar, a.err);
+  const bool skip = *ctx.abort_flag != 0;
+  const int warp = static_cast<int>(threadIdx.x >> 5), lane = static_cast<int>(threadIdx.x & 31);
+  const int S = a.seqlen, W = a.window;
+  // longest first: query tiles from the end of the sequence
+  const int per_tile = kNumKvHeads * a.batch;
+  const int idx = static_cast<int>(blockIdx.x);
+  const int qt = a.n_qt - 1 - idx / per_tile;
+  const int g = (idx % per_tile) % kNumKvHeads, b = (idx % per_tile) / kNumKvHeads;
+  const int q0 = qt * kTok;
+  const int tlast = min(q0 + kTok - 1, S - 1);
+  const int jt0 = W > 0 ? max(0, q0 - W + 1) / kKeys : 0;
+  const int n_tiles = tlast / kKeys - jt0 + 1;
+
+  if (warp == 0) {
+    if (lane == 0 && !skip) {
+      prefetch_tensormap(&maps.q);
+      prefetch_tensormap(&maps.dout);
+      prefetch_tensormap(&maps.k);
+      prefetch_tensormap(&maps.v);
+      mbar_arrive_expect_tx(ctx.bar(BAR_Q_FULL), 2 * kTile);
+      tma_load_4d(ctx.sbase + kQOffQ, &maps.q, ctx.bar(BAR_Q_FULL), 0, g * kGroup, q0, b);
+      tma_load_4d(ctx.sbase + kQOffDO, &maps.dout, ctx.bar(BAR_Q_FULL), 0, g * kGroup, q0, b);
+      int j = 0;
+      for (; j < n_tiles; ++j) {
+        const int s = j % kStages;
+        if (j >= kStages && !ctx.wait(BAR_KV_EMPTY + s, ((j / kStages) - 1) & 1)) break;
+        mbar_arrive_expect_tx(ctx.bar(BAR_KV_FULL + s), 2 * kTile);
+        tma_load_4d(ctx.sbase + kQOffK + s * kTile, &maps.k, ctx.bar(BAR_KV_FULL + s), 0, g,
+                    (jt0 + j) * kKeys, b);
+        tma_load_4d(ctx.sbase + kQOffV + s * kTile, &maps.v, ctx.bar(BAR_KV_FULL + s), 0, g,
+                    (jt0 + j) * kKeys, b);
+      }
+      if (*ctx.abort_flag) {
+        volatile int never = 0;
+        mbar_wait(ctx.bar(BAR_Q_FULL), 0, &never, nullptr, 0, kWaitTimeoutNs);
+        for (int i = max(0, j - kStages); i < j; ++i)
+          mbar_wait(ctx.bar(BAR_KV_FULL + i % kStages), (i / kStages) & 1, &never, nullptr, 0,
+                    kWaitTimeoutNs);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && !skip) {
+      bool ok = ctx.wait(BAR_Q_FULL, 0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kStages;
+        if (!(ok = ctx.wait(BAR_KV_FULL + s, (j / kStages) & 1))) break;
+        // the elementwise warps have read S and dP of the previous tile (and
+        // dQ of that tile, issued before, reads dS first: one thread's MMAs
+        // run in order)
+        if (j > 0 && !(ok = ctx.wait(BAR_E_DONE, (j - 1) & 1))) break;
+        tc_fence_after_sync();
+        if (j > 0) {
+          const int sp = (j - 1) % kStages;
+          mma_tmem_a(tmem + kColA, tmem + kColS, ctx.sbase + kQOffK + sp * kTile, j > 1);
+          mma_commit(ctx.bar(BAR_KV_EMPTY + sp));
+        }
+        mma_abt(tmem + kColS, ctx.sbase + kQOffQ, ctx.sbase + kQOffK + s * kTile);
+        mma_abt(tmem + kColP, ctx.sbase + kQOffDO, ctx.sbase + kQOffV + s * kTile);
+        mma_commit(ctx.bar(BAR_S_FULL));
+      }
+      if (ok && (ok = ctx.wait(BAR_E_DONE, (n_tiles - 1) & 1))) {
+        tc_fence_after_sync();
+        const int sp = (n_tiles - 1) % kStages;
+        mma_tmem_a(tmem + kColA, tmem + kColS, ctx.sbase + kQOffK + sp * kTile, n_tiles > 1);
+        mma_commit(ctx.bar(BAR_KV_EMPTY + sp));
+        mma_commit(ctx.bar(BAR_ACC_FULL));
+      }
+      mma_commit(ctx.bar(BAR_MMA_DONE));
+      volatile int never = 0;
+      mbar_wait(ctx.bar(BAR_MMA_DONE), 0, &never, nullptr, 0, kWaitTimeoutNs);
+    }
+  } else if (warp >= 4) {
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // row: token q0 + r/8, head g*8 + r%8
+    const int t = q0 + (r >> 3);
+    const bool row_ok = t < S;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    float lse2 = 0.f, dd = 0.f;
+    if (row_ok) {
+      const int64_t w = ((static_cast<int64_t>(b) * kNumKvHeads + g) * S + t) * kGroup + (r & 7);
+      lse2 = a.lse2[w];
+      dd = a.dd[w];
+    }
+    bool ok = !skip;
+    for (int j = 0; ok && j < n_tiles; ++j) {
+      if (!(ok = ctx.wait_warp(BAR_S_FULL, j & 1))) break;
+      tc_fence_after_sync();
+      const int kb = (jt0 + j) * kKeys;
+      const int c_hi = t - kb;                           // visible columns [c_lo, c_hi]
+      const int c_lo = W > 0 ? t - W + 1 - kb : -1;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], pv[32], out[16];
+        tmem_ld32(tmem + lane_off + kColS + 32 * c, sv);
+        tmem_ld32(tmem + lane_off + kColP + 32 * c, pv);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int col = 32 * c + e + u;
+            const bool vis = row_ok && col <= c_hi && col >= c_lo;
+            const float p = vis ? ex2_approx(__uint_as_float(sv[e + u]) * kScaleLog2 - lse2) : 0.f;
+            ds[u] = p * (__uint_as_float(pv[e + u]) - dd) * kScale;
+          }
+          out[e / 2] = pack_bf16x2(ds[0], ds[1]);
+        }
+        // dS (bf16 pairs) into S's columns [16c, 16c+16), all of which were read already
+        tmem_st16(tmem + lane_off + kColS + 16 * c, out);
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ctx.bar(BAR_E_DONE));
+    }
+    if (ok && (ok = ctx.wait_warp(BAR_ACC_FULL, 0))) {
+      tc_fence_after_sync();
+      uint32_t lo[32], hi[32];
+      tmem_ld32(tmem + lane_off + kColA, lo);
+      tmem_ld32(tmem + lane_off + kColA + 32, hi);
+      if (row_ok) {
+        const int p = bwd::clamp_pos(__ldg(a.pos + static_cast<int64_t>(b) * S + t), a.err);
+        unrotate_store(lo, hi, a.rope + static_cast<size_t>(p) * kRopePairs,
+                       a.dq + ((static_cast<int64_t>(b) * S + t) * kNumHeads + g * kGroup +
+                               (r & 7)) * kHeadDim);
+      }
+    }
+  }
+  teardown(tmem);
+}
+
+// dK and dV for one (b, g, 128-key) tile per CTA.
+__global__ void __launch_bounds__(bwd::kThreads, 1)
+    bwd_dkv_kernel(const __grid_constant__ BackwardMaps maps, const BackwardArgs a) {
+  using namespace bwd;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  Ctx ctx;
+  const uint32_t tmem = setup(ctx, smem, kKOffBar, a.err);
+  const bool skip = *ctx.abort_flag != 0;
+  const int warp = static_cast<int>(threadIdx.x >> 5), lane = static_cast<int>(threadIdx.x & 31);
+  const int S = a.seqlen, W = a.window;
+  // longest first: key tiles from the start of the sequence
+  const int per_tile = kNumKvHeads * a.batch;
+  const int idx = static_cast<int>(blockIdx.x);
+  const int kt = idx / per_tile;
+  const int g = (idx % per_tile) % kNumKvHeads, b = (idx % per_tile) / kNumKvHeads;
+  const int kb = kt * kKeys;
+  // query tokens that see a key of this tile: [kb, t_max]
+  const int t_max = W > 0 ? min(S - 1, kb + kKeys - 1 + W - 1) : S - 1;
+  const int qt0 = kb / kTok;
+  const int n_tiles = t_max / kTok - qt0 + 1;
+  const float* lse2_g = a.lse2 + (static_cast<int64_t>(b) * kNumKvHeads + g) * S * kGroup;
+  const float* dd_g = a.dd + (static_cast<int64_t>(b) * kNumKvHeads + g) * S * kGroup;
+
+  if (warp == 0) {
+    if (lane == 0 && !skip) {
+      prefetch_tensormap(&maps.q);
+      prefetch_tensormap(&maps.dout);
+      prefetch_tensormap(&maps.k);
+      prefetch_tensormap(&maps.v);
+      mbar_arrive_expect_tx(ctx.bar(BAR_KV_FULL), 2 * kTile);
+      tma_load_4d(ctx.sbase + kKOffK, &maps.k, ctx.bar(BAR_KV_FULL), 0, g, kb, b);
+      tma_load_4d(ctx.sbase + kKOffV, &maps.v, ctx.bar(BAR_KV_FULL), 0, g, kb, b);
+      int j = 0;
+      for (; j < n_tiles; ++j) {
+        const int s = j % kStages;
+        if (j >= kStages && !ctx.wait(BAR_Q_EMPTY + s, ((j / kStages) - 1) & 1)) break;
+        const int t0 = (qt0 + j) * kTok;
+        const uint32_t st = ctx.sbase + kKOffQ + s * 2 * kTile;
+        const uint32_t ld = ctx.sbase + kKOffLD + s * 1024;
+        // lse2 and D of the tile's 128 rows: 512 contiguous bytes each (the
+        // arrays are padded by one tile, rows past the sequence are masked)
+        mbar_arrive_expect_tx(ctx.bar(BAR_Q_FULL + s), 2 * kTile + 1024);
+        tma_load_4d(st, &maps.q, ctx.bar(BAR_Q_FULL + s), 0, g * kGroup, t0, b);
+        tma_load_4d(st + kTile, &maps.dout, ctx.bar(BAR_Q_FULL + s), 0, g * kGroup, t0, b);
+        bulk_load(ld, lse2_g + static_cast<int64_t>(t0) * kGroup, 512, ctx.bar(BAR_Q_FULL + s));
+        bulk_load(ld + 512, dd_g + static_cast<int64_t>(t0) * kGroup, 512,
+                  ctx.bar(BAR_Q_FULL + s));
+      }
+      if (*ctx.abort_flag) {
+        volatile int never = 0;
+        mbar_wait(ctx.bar(BAR_KV_FULL), 0, &never, nullptr, 0, kWaitTimeoutNs);
+        for (int i = max(0, j - kStages); i < j; ++i)
+          mbar_wait(ctx.bar(BAR_Q_FULL + i % kStages), (i / kStages) & 1, &never, nullptr, 0,
+                    kWaitTimeoutNs);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && !skip) {
+      bool ok = ctx.wait(BAR_KV_FULL, 0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kStages;
+        if (!(ok = ctx.wait(BAR_Q_FULL + s, (j / kStages) & 1))) break;
+        if (j > 0 && !(ok = ctx.wait(BAR_E_DONE, (j - 1) & 1))) break;
+        tc_fence_after_sync();
+        if (j > 0) {
+          const int sp = (j - 1) % kStages;
+          const uint32_t st = ctx.sbase + kKOffQ + sp * 2 * kTile;
+          mma_tmem_a(tmem + kColA, tmem + kColS, st + kTile, j > 1);  // dV += P^T dO
+          mma_tmem_a(tmem + kColB, tmem + kColP, st, j > 1);          // dK += dS^T Q'
+          mma_commit(ctx.bar(BAR_Q_EMPTY + sp));
+        }
+        const uint32_t st = ctx.sbase + kKOffQ + s * 2 * kTile;
+        mma_abt(tmem + kColS, ctx.sbase + kKOffK, st);           // S^T = K' Q'^T
+        mma_abt(tmem + kColP, ctx.sbase + kKOffV, st + kTile);   // dP^T = V dO^T
+        mma_commit(ctx.bar(BAR_S_FULL));
+      }
+      if (ok && (ok = ctx.wait(BAR_E_DONE, (n_tiles - 1) & 1))) {
+        tc_fence_after_sync();
+        const int sp = (n_tiles - 1) % kStages;
+        const uint32_t st = ctx.sbase + kKOffQ + sp * 2 * kTile;
+        mma_tmem_a(tmem + kColA, tmem + kColS, st + kTile, n_tiles > 1);
+        mma_tmem_a(tmem + kColB, tmem + kColP, st, n_tiles > 1);
+        mma_commit(ctx.bar(BAR_Q_EMPTY + sp));
+        mma_commit(ctx.bar(BAR_ACC_FULL));
+      }
+      mma_commit(ctx.bar(BAR_MMA_DONE));
+      volatile int never = 0;
+      mbar_wait(ctx.bar(BAR_MMA_DONE), 0, &never, nullptr, 0, kWaitTimeoutNs);
+    }
+  } else if (warp >= 4) {
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // key kb + r
+    const int kj = kb + r;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    bool ok = !skip;
+    for (int j = 0; ok && j < n_tiles; ++j) {
+      const int s = j % kStages;
+      if (!(ok = ctx.wait_warp(BAR_S_FULL, j & 1))) break;
+      tc_fence_after_sync();
+      const int t0 = (qt0 + j) * kTok;
+      const float* ld = reinterpret_cast<const float*>(smem + kKOffLD + s * 1024);
+      // column col is token t0 + col/8: visible iff kj <= t < S and t < kj + W
+      const int lo_t = kj - t0;                              // first visible token offset
+      const int hi_t = min(S - 1 - t0, W > 0 ? kj + W - 1 - t0 : 1 << 30);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], pv[32], pw[16], dw[16];
+        tmem_ld32(tmem + lane_off + kColS + 32 * c, sv);
+        tmem_ld32(tmem + lane_off + kColP + 32 * c, pv);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float p[2], ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int col = 32 * c + e + u;
+            const int tt = col >> 3;
+            const bool vis = tt >= lo_t && tt <= hi_t;
+            p[u] = vis ? ex2_approx(__uint_as_float(sv[e + u]) * kScaleLog2 - ld[col]) : 0.f;
+            ds[u] = p[u] * (__uint_as_float(pv[e + u]) - ld[128 + col]) * kScale;
+          }
+          pw[e / 2] = pack_bf16x2(p[0], p[1]);
+          dw[e / 2] = pack_bf16x2(ds[0], ds[1]);
+        }
+        tmem_st16(tmem + lane_off + kColS + 16 * c, pw);
+        tmem_st16(tmem + lane_off + kColP + 16 * c, dw);
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ctx.bar(BAR_E_DONE));
+    }
+    if (ok && (ok = ctx.wait_warp(BAR_ACC_FULL, 0))) {
+      tc_fence_after_sync();
+      uint32_t lo[32], hi[32];
+      tmem_ld32(tmem + lane_off + kColA, lo);
+      tmem_ld32(tmem + lane_off + kColA + 32, hi);
+      if (kj < S) {
+        uint4* dv4 = reinterpret_cast<uint4*>(
+            a.dv + ((static_cast<int64_t>(b) * S + kj) * kNumKvHeads + g) * kHeadDim);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          dv4[i] = make_uint4(pack_bf16x2(__uint_as_float(lo[8 * i]), __uint_as_float(lo[8 * i + 1])),
+                              pack_bf16x2(__uint_as_float(lo[8 * i + 2]), __uint_as_float(lo[8 * i + 3])),
+                              pack_bf16x2(__uint_as_float(lo[8 * i + 4]), __uint_as_float(lo[8 * i + 5])),
+                              pack_bf16x2(__uint_as_float(lo[8 * i + 6]), __uint_as_float(lo[8 * i + 7])));
+          dv4[4 + i] = make_uint4(pack_bf16x2(__uint_as_float(hi[8 * i]), __uint_as_float(hi[8 * i + 1])),
+                                  pack_bf16x2(__uint_as_float(hi[8 * i + 2]), __uint_as_float(hi[8 * i + 3])),
+                                  pack_bf16x2(__uint_as_float(hi[8 * i + 4]), __uint_as_float(hi[8 * i + 5])),
+                                  pack_bf16x2(__uint_as_float(hi[8 * i + 6]), __uint_as_float(hi[8 * i + 7])));
+        }
+      }
+      tmem_ld32(tmem + lane_off + kColB, lo);
+      tmem_ld32(tmem + lane_off + kColB + 32, hi);
+      if (kj < S) {
+        const int p = bwd::clamp_pos(__ldg(a.pos + static_cast<int64_t>(b) * S + kj), a.err);
+        unrotate_store(lo, hi, a.rope + static_cast<size_t>(p) * kRopePairs,
+                       a.dk + ((static_cast<int64_t>(b) * S + kj) * kNumKvHeads + g) * kHeadDim);
+      }
+    }
+  }
+  teardown(tmem);
+}
+
+}  // namespace
+
+int backward_q_tiles(int seqlen) { return (seqlen + bwd::kTok - 1) / bwd::kTok; }
+int backward_k_tiles(int seqlen) { return (seqlen + bwd::kKeys - 1) / bwd::kKeys; }
+
+cudaError_t launch_backward(const BackwardMaps& maps, const BackwardArgs& args, int num_sms,
+                            cudaStream_t stream) {
+  const int64_t ntok = static_cast<int64_t>(args.batch) * args.seqlen;
+  int64_t prep_blocks = (ntok + 3) / 4;
+  if (prep_blocks > 4 * num_sms) prep_blocks = 4 * num_sms;
+  bwd_prep_kernel<<<static_cast<unsigned>(prep_blocks), 256, 0, stream>>>(args);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bwd::kSmemBytes));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bwd::kSmemBytes));
+  if (e != cudaSuccess) return e;
+  const unsigned n_dq = static_cast<unsigned>(args.n_qt * kNumKvHeads * args.batch);
+  bwd_dq_kernel<<<n_dq, bwd::kThreads, bwd::kSmemBytes, stream>>>(maps, args);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const unsigned n_dkv =
+      static_cast<unsigned>(backward_k_tiles(args.seqlen) * kNumKvHeads * args.batch);
+  bwd_dkv_kernel<<<n_dkv, bwd::kThreads, bwd::kSmemBytes, stream>>>(maps, args);
+  return cudaGetLastError();
+}
+
+}  // namespace gqa

@@ -91,6 +91,7 @@ extern "C" int gptoss_attn_decode_noalloc(const void* q, const void* kcache, con
   a.vcache = static_cast<const uint16_t*>(vcache);
   a.sinks = sinks;
   a.len = len;
+  a.rope = nullptr;  // plain RoPE, evaluated in the kernel
   a.out = static_cast<uint16_t*>(out);
   const size_t rows = static_cast<size_t>(batch) * kNumHeads * nsplit;
   a.part_o = reinterpret_cast<float*>(scratch + kErrBytes);

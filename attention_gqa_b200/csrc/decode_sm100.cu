@@ -134,11 +134,18 @@ __global__ void __launch_bounds__(kThreads)
   // rotation of the new query at position L-1 (fp64 angles)
   float2* cs = reinterpret_cast<float2*>(smem + kOffCS);
   if (t < kRopePairs) {
-    const double ang = static_cast<double>(L > 0 ? L - 1 : 0) *
-                       pow(kRopeTheta, -2.0 * static_cast<double>(t) / kHeadDim);
-    double sn, cn;
-    sincos(ang, &sn, &cn);
-    cs[t] = make_float2(static_cast<float>(cn), static_cast<float>(sn));
+    if (a.rope) {
+      // a table (YaRN) covers positions below kMaxPosition; the API limits
+      // max_len to that, and len is clamped to max_len above
+      const int p = min(L > 0 ? L - 1 : 0, kMaxPosition - 1);
+      cs[t] = a.rope[static_cast<size_t>(p) * kRopePairs + t];
+    } else {
+      const double ang = static_cast<double>(L > 0 ? L - 1 : 0) *
+                         pow(kRopeTheta, -2.0 * static_cast<double>(t) / kHeadDim);
+      double sn, cn;
+      sincos(ang, &sn, &cn);
+      cs[t] = make_float2(static_cast<float>(cn), static_cast<float>(sn));
+    }
   }
   named_barrier(1, kWarps * 32);
   uint16_t* qs = reinterpret_cast<uint16_t*>(smem + kOffQ);

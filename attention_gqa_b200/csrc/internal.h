@@ -29,6 +29,8 @@ struct PrefillArgs {
   const float* sinks;   // [64]
   const float2* rope;   // [kMaxPosition][32] (cos, sin)
   int* err;             // device error word
+  float* lse;           // [B][S][64] natural-log softmax normaliser per row (sink
+                        // included), written when not null; indexed like out
   int batch;
   int seqlen;           // query tokens per sequence (the rows of q, pos and out)
   int q_start;          // key index of query token 0: keys come from a cache
@@ -55,8 +57,9 @@ cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cud
 // Diagnostic: a bounded wait on a barrier nothing arrives at (sets kErrTimeout).
 cudaError_t launch_wait_timeout(int* err, uint64_t timeout_ns, cudaStream_t stream);
 
-// Fills the rotary table [kMaxPosition][32] of (cos, sin).
-cudaError_t launch_rope_table(float2* table, cudaStream_t stream);
+// Fills the rotary table [kMaxPosition][32] of (cos, sin); with `yarn` the
+// YaRN frequencies and attention factor of the model.
+cudaError_t launch_rope_table(float2* table, bool yarn, cudaStream_t stream);
 
 // Rotates the rows of x [batch][n][heads][64] (bf16; heads = 8 for keys or 64
 // for queries) by pos[batch][n] into x_rot laid out [batch][dst_len][heads][64],
@@ -71,6 +74,8 @@ struct DecodeArgs {
   const uint16_t* vcache;  // [B][L][8][64] bf16
   const float* sinks;      // [64]
   const int32_t* len;      // [B]
+  const float2* rope;      // rotary table rows for the query, or nullptr: plain RoPE
+                           // evaluated in fp64 in the kernel
   uint16_t* out;           // [B][64][64] bf16
   float* part_o;           // [B][64][nsplit][64]
   float2* part_ml;         // [B][64][nsplit] (max in log2 units, sum)
@@ -87,6 +92,38 @@ struct DecodeMaps {
 };
 
 cudaError_t launch_decode(const DecodeMaps& maps, const DecodeArgs& args, cudaStream_t stream);
+
+struct BackwardArgs {
+  const int32_t* pos;      // [B][S]
+  const float* sinks;      // [64]
+  const float2* rope;      // rotary table
+  int* err;
+  const float* lse;        // [B][S][64] from the forward (natural log)
+  const uint16_t* out;     // [B][S][64][64] bf16, the forward output
+  const uint16_t* dout;    // [B][S][64][64] bf16
+  float* lse2;             // workspace [B][8][S][8] (+ one tile of padding), log2 units
+  float* dd;               // workspace [B][8][S][8] (+ padding): dO . out per row
+  float* dsinks;           // [64], zeroed before the launch
+  uint16_t* dq;            // [B][S][64][64] bf16
+  uint16_t* dk;            // [B][S][8][64] bf16
+  uint16_t* dv;            // [B][S][8][64] bf16
+  int batch;
+  int seqlen;
+  int window;              // <= 0: full causal
+  int n_qt;                // 16-token query tiles per sequence
+};
+
+struct BackwardMaps {
+  CUtensorMap q, dout;     // rotated q and dO: boxes (64, 8, 16, 1)
+  CUtensorMap k, v;        // rotated k and v: boxes (64, 1, 128, 1)
+};
+
+int backward_q_tiles(int seqlen);
+int backward_k_tiles(int seqlen);
+// Launches the preparation, dQ and dK/dV kernels (dsinks must be zeroed and
+// the rotated q and k written to the workspace before).
+cudaError_t launch_backward(const BackwardMaps& maps, const BackwardArgs& args, int num_sms,
+                            cudaStream_t stream);
 
 // Decode split planning shared by the workspace query and the launch.
 void decode_plan(int batch, int max_len, int window, int* nsplit, int* chunk);

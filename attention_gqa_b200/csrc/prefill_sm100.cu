@@ -71,6 +71,7 @@ constexpr uint32_t kRegsSoftmax = 184;  // WG1 and WG2
 static_assert(2 * 128 * kRegsLight + 2 * 128 * kRegsSoftmax <= 512 * 128, "register split");
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kScaleLog2 = 0.125f * kLog2e;  // 1/sqrt(64) * log2(e)
 constexpr float kRescaleThreshold = 8.0f;      // log2 units
 // Exp-loop step (of 64 column pairs) at which a softmax warpgroup releases the
@@ -222,10 +223,6 @@ __device__ __forceinline__ uint32_t stage_rope_rows(const PrefillArgs& a, int b,
     }
   }
   return bytes;
-}
-
-__device__ __forceinline__ bool key_visible(int kj, int tq, int W) {
-  return kj <= tq && (W <= 0 || kj > tq - W);
 }
 
 // S_m = Q_m K^T for one K/V tile (4 MMAs of K = 16 over head_dim 64).
@@ -467,9 +464,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kb = (it.jt0 + j) * kBlockN;
         const bool wmask = (kb + kBlockN - 1 > tmin) || (W > 0 && kb <= tmax - W);
         if (wmask) {
+          // this row sees the tile's columns [c_lo, c_hi] (keys tq-W < j <= tq)
+          const int c_hi = tq - kb;
+          const int c_lo = W > 0 ? tq - W + 1 - kb : -1;
 #pragma unroll
           for (int i = 0; i < 128; ++i)
-            if (!key_visible(kb + i, tq, W)) sv[i] = __float_as_uint(-INFINITY);
+            if (i > c_hi || i < c_lo) sv[i] = __float_as_uint(-INFINITY);
         }
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
@@ -564,6 +564,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = ctx.wait_warp(BAR_O_FULL + m, n & 1))) break;
       tc_fence_after_sync();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      if (args.lse) {
+        // natural-log normaliser of this row: (m_ref + log2 l) ln 2
+        const int t = it.q0 + m * kTokensPerM + (r >> 3);
+        if (t < S)
+          args.lse[(static_cast<size_t>(it.b) * S + t) * kNumHeads + it.g * kGroup + (r & 7)] =
+              l > 0.f ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
+      }
       uint8_t* stage = smem + kOffQ + (2 * qs + m) * kTileBytes;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -981,6 +988,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         l0 = a0 + a2;
         l1 = a1 + a3;
       }
+      if (args.lse && it.q0 + d < S)
+        args.lse[(static_cast<size_t>(it.b) * S + it.q0 + d) * kNumHeads + it.g * kGroup +
+                 (r & 7)] = (mr + __log2f(l0 + l1)) * kLn2;
       {
         uint32_t a[64], b8[8];
 #pragma unroll

@@ -5,6 +5,14 @@
 // rope_table_kernel: for every position p < 131072 and pair k < 32 the
 //   (cos, sin) of p * theta^(-2k/64). Angles reach 1.3e5 rad, so they are
 //   formed and reduced in fp64; only the results are stored as fp32.
+//   The YaRN table (techniques map row "YaRN RoPE scaling": factor 32 over the
+//   4096-token initial context of the llm-atlas field tables) blends each
+//   pair's frequency between theta^(-2k/64) and theta^(-2k/64) / 32 by a ramp
+//   linear in the pair index, from 0 at the pair whose wavelength fits 32 times
+//   into 4096 tokens to 1 at the pair where it fits once (the transformers yarn
+//   initialisation, beta_fast 32 and beta_slow 1, no truncation), and scales
+//   cos and sin by the attention factor 0.1 ln 32 + 1, which therefore reaches
+//   both the rotated queries and the rotated keys.
 // rope_rows_kernel: rotates every key row once per layer into a workspace,
 //   so the attention kernels, which read each key tile many times, never
 //   rotate keys. HBM bound: 128 bytes read and written per row.
@@ -14,15 +22,34 @@
 namespace gqa {
 namespace {
 
-__global__ void rope_table_kernel(float2* __restrict__ table) {
+constexpr double kYarnFactor = 32.0;
+constexpr double kYarnContext = 4096.0;
+constexpr double kYarnTurnsFast = 32.0;  // beta_fast: full turns over the context
+constexpr double kYarnTurnsSlow = 1.0;   // beta_slow
+constexpr double kTwoPi = 6.283185307179586476925286766559;
+
+// Pair index (fractional) at which theta^(-2k/64) * context / (2 pi) = turns.
+__device__ double yarn_pair(double turns) {
+  return kHeadDim * log(kYarnContext / (turns * kTwoPi)) / (2.0 * log(kRopeTheta));
+}
+
+__global__ void rope_table_kernel(float2* __restrict__ table, int yarn) {
   const int idx = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
   if (idx >= kMaxPosition * kRopePairs) return;
   const int p = idx / kRopePairs;
   const int k = idx % kRopePairs;
-  const double inv_freq = pow(kRopeTheta, -2.0 * static_cast<double>(k) / kHeadDim);
+  double inv_freq = pow(kRopeTheta, -2.0 * static_cast<double>(k) / kHeadDim);
+  double scale = 1.0;
+  if (yarn) {
+    const double lo = fmax(yarn_pair(kYarnTurnsFast), 0.0);
+    const double hi = fmin(yarn_pair(kYarnTurnsSlow), kHeadDim - 1.0);
+    const double w = fmin(fmax((static_cast<double>(k) - lo) / (hi - lo), 0.0), 1.0);
+    inv_freq = w * (inv_freq / kYarnFactor) + (1.0 - w) * inv_freq;
+    scale = 0.1 * log(kYarnFactor) + 1.0;
+  }
   double s, c;
   sincos(static_cast<double>(p) * inv_freq, &s, &c);
-  table[idx] = make_float2(static_cast<float>(c), static_cast<float>(s));
+  table[idx] = make_float2(static_cast<float>(c * scale), static_cast<float>(s * scale));
 }
 
 // Four threads per 64-element row; thread c rotates the 16-byte chunks c and
@@ -100,9 +127,9 @@ cudaError_t launch_wait_timeout(int* err, uint64_t timeout_ns, cudaStream_t stre
   return cudaGetLastError();
 }
 
-cudaError_t launch_rope_table(float2* table, cudaStream_t stream) {
+cudaError_t launch_rope_table(float2* table, bool yarn, cudaStream_t stream) {
   const int n = kMaxPosition * kRopePairs;
-  rope_table_kernel<<<(n + 255) / 256, 256, 0, stream>>>(table);
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, stream>>>(table, yarn ? 1 : 0);
   return cudaGetLastError();
 }
 

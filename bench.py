@@ -1,26 +1,33 @@
 """Throughput of the gpt-oss attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload step|tiny256|batch16k|seq128k|layers36|chunk16k]
+                    [--workload default|s4096|tiny256|batch16k|layers36|chunk16k]
 
-One step is one pass of the whole path over one batch of synthetic inputs:
-  * prefill, B=1, S=4096, 64 query / 8 key-value heads, head_dim 64: a
-    128-token sliding-window layer, then a full-causal layer, each with its
-    own seeded q/k/v/sinks (RoPE table, rotation, QK^T, sink-seeded online
-    softmax, PV, epilogue);
+One step is one pass of the whole path over one batch of synthetic inputs. The
+default workload is the largest single-GPU configuration:
+  * prefill, B=1, S=131072, 64 query / 8 key-value heads, head_dim 64: one
+    full-causal layer and one 128-token sliding-window layer, each with its
+    own seeded q/k/v/sinks (key rotation, then the attention kernel: Q
+    rotation, QK^T, sink-seeded online softmax, PV, epilogue);
   * decode, B=64 sequences against a bf16 cache of 8192 tokens: one
     full-causal layer and one sliding layer (its last 128 entries)
     (split-KV partials + log-sum-exp combine).
-``value`` is the prefill attention throughput in TFLOP/s counting unmasked
-FLOPs only (4 * 64 * 64 per visible (query, key) pair per head); the decode
-half of the metric (HBM GB/s over the algorithmic bytes) is reported in the
-``decode`` object. L2 is flushed (256 MB write) before every step, outside
-the timed events. Per-kernel times come from CUDA events on the launching
-stream. With N > 1 (torchrun), every rank runs the same per-GPU workload
-(weak scaling, no collective on the data path); times are the max over ranks.
+``--workload s4096`` runs the same step with a B=1, S=4096 prefill (a W=128
+layer, then a full-causal layer). ``value`` is the prefill attention
+throughput in TFLOP/s counting unmasked FLOPs only (4 * 64 * 64 per visible
+(query, key) pair per head); the decode half of the metric (HBM GB/s over the
+algorithmic bytes) is reported in the ``decode`` object. L2 is flushed (256 MB
+write) before every step, outside the timed events. Per-kernel times come from
+CUDA events on the launching stream. With N > 1 (torchrun), every rank runs
+the same per-GPU workload (weak scaling, no collective on the data path);
+times are the max over ranks.
 
-``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
-same workload (rank 0 only).
+Inputs follow the seeded recipe of ``synth`` (SplitMix64 -> Box-Muller ->
+fp32 -> bf16), evaluated on the device by ``synth.device``.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores, rank 0 only:
+each step is one bounded sample of the same workload (evenly spaced query rows
+of both prefill layers, a few decode sequences of both decode layers).
 """
 from __future__ import annotations
 
@@ -41,13 +48,22 @@ import numpy as np  # noqa: E402
 
 METRIC = "attention TFLOP/s (unmasked) & % bf16 peak; decode HBM GB/s & % of peak"
 NQ, NKV, D = 64, 8, 64
-PREFILL_B, PREFILL_S = 1, 4096
-PREFILL_LAYERS = ((0, 128), (1, 0))          # (layer index, window): sliding then full
-DECODE_B, DECODE_L = 64, 8192
-DECODE_LAYERS = ((0, 0), (1, 128))            # full, then sliding
-WORKLOAD = ("prefill B=1 S=4096 64q/8kv d64 (W=128 layer + full-causal layer) + "
-            "decode B=64 L=8192 (full layer + W=128 layer)")
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "prefill_full_S4096_traffic.txt")
+
+# A step workload: a prefill of B x S tokens through `pre_layers` [(layer, window)]
+# with the seeds of configuration `pre_cfg`, then decode of DB sequences against
+# DL cached tokens through `dec_layers` with the seeds of configuration `dec_cfg`.
+STEP_WORKLOADS = {
+    "default": dict(
+        pre_cfg=5, B=1, S=131072, pre_layers=((0, 0), (1, 128)),
+        dec_cfg=4, DB=64, DL=8192, dec_layers=((0, 0), (1, 128)), peak="sustained",
+        desc="prefill B=1 S=131072 64q/8kv d64 (one full-causal layer + one W=128 layer) + "
+             "decode B=64 L=8192 (one full layer + one W=128 layer)"),
+    "s4096": dict(
+        pre_cfg=2, B=1, S=4096, pre_layers=((0, 128), (1, 0)),
+        dec_cfg=4, DB=64, DL=8192, dec_layers=((0, 0), (1, 128)), peak="burst",
+        desc="prefill B=1 S=4096 64q/8kv d64 (W=128 layer + full-causal layer) + "
+             "decode B=64 L=8192 (full layer + W=128 layer)"),
+}
 
 
 def visible_pairs(S: int, window: int) -> int:
@@ -86,12 +102,12 @@ def source_digest() -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per launch of the full-causal prefill kernel from the committed
+def profiled_traffic(path: str):
+    """DRAM bytes per launch of the full-causal prefill kernel from a committed
     ncu summary, if it was taken on the current kernel source."""
     try:
         vals = {}
-        with open(PROFILE_TRAFFIC) as f:
+        with open(path) as f:
             for line in f:
                 if ":" in line and not line.startswith("#"):
                     k, v = line.split(":", 1)
@@ -160,52 +176,161 @@ def host_cores() -> int:
         return os.cpu_count() or 1
 
 
+def step_config(wl: dict) -> dict:
+    """The workload description both arms print (identical, so the lines compare)."""
+    return {"workload": wl["desc"], "prefill": {"batch": wl["B"], "seq_len": wl["S"],
+                                                "windows": [w for _, w in wl["pre_layers"]]},
+            "decode": {"batch": wl["DB"], "cache_len": wl["DL"],
+                       "windows": [w for _, w in wl["dec_layers"]]},
+            "l2": "flushed before every step (256 MB write)"}
+
+
 # ------------------------------------------------------------------ CPU oracle leg
 
-def oracle_sample(budget_s: float = 12.0):
-    """Times the fp64 oracle on evenly spaced query rows of the two prefill
-    layers (all 64 heads of each row); returns (TFLOP/s, seconds, rows, FLOPs)."""
-    import oracle
+def _seed(cfg, layer, tid):
     import synth
-    oracle._load()
-    total_flops, total_s, nrows = 0.0, 0.0, 0
-    per_layer = budget_s / len(PREFILL_LAYERS)
-    for layer, window in PREFILL_LAYERS:
-        x = synth.make_prefill_inputs(2, layer, PREFILL_B, PREFILL_S)
-        k = synth.bf16_bits_to_f64(x["k"])
-        v = synth.bf16_bits_to_f64(x["v"])
-        n = 64
-        while True:
-            toks = np.linspace(0, PREFILL_S - 1, n).astype(np.int64)
-            rows = [(0, int(t)) for t in toks]
-            q_rows = synth.bf16_bits_to_f64(np.stack([x["q"][0, t] for t in toks]))
+    return synth.seed_for(cfg, layer, tid)
+
+
+class OracleSampler:
+    """Bounded samples of a step workload for the fp64 CPU oracle.
+
+    Holds, on the host, the keys and values of every prefill layer and of a few
+    decode sequences per decode layer (same seeded recipe as the GPU arm). One
+    sample is: `rows` evenly spaced query rows (all 64 heads) of each prefill
+    layer, shifted by the sample index, and `seqs` decode sequences of each
+    decode layer."""
+
+    def __init__(self, wl: dict, tensors=None, n_seqs: int = 2):
+        import torch
+
+        import synth
+        from synth import device as sdev
+        self.wl = wl
+        B, S = wl["B"], wl["S"]
+        self.pre = []
+        for i, (layer, window) in enumerate(wl["pre_layers"]):
+            if tensors is not None:
+                t = tensors["pre"][i]
+                k, v, sinks = (t["k"].double().cpu().numpy(), t["v"].double().cpu().numpy(),
+                               t["sinks"].double().cpu().numpy())
+            else:
+                k = sdev.bf16_normal(_seed(wl["pre_cfg"], layer, synth.TENSOR_K),
+                                     (B, S, NKV, D), "cpu").double().numpy()
+                v = sdev.bf16_normal(_seed(wl["pre_cfg"], layer, synth.TENSOR_V),
+                                     (B, S, NKV, D), "cpu").double().numpy()
+                sinks = sdev.f32_normal(_seed(wl["pre_cfg"], layer, synth.TENSOR_SINKS), (NQ,),
+                                        "cpu").double().numpy()
+            pos = np.broadcast_to(np.arange(S, dtype=np.int32), (B, S)).copy()
+            self.pre.append(dict(layer=layer, window=window, k=k, v=v, sinks=sinks, pos=pos))
+        DB, DL = wl["DB"], wl["DL"]
+        self.n_seqs = min(n_seqs, DB)
+        self.dec = []
+        per_seq = DL * NKV * D
+        for layer, window in wl["dec_layers"]:
+            qseed = _seed(wl["dec_cfg"], layer, synth.TENSOR_Q)
+            kseed = _seed(wl["dec_cfg"], layer, synth.TENSOR_K)
+            vseed = _seed(wl["dec_cfg"], layer, synth.TENSOR_V)
+            def rows(seed, n):
+                return torch.stack([sdev.bf16_normal_range(seed, i * n, n, "cpu")
+                                    for i in range(self.n_seqs)]).double().numpy()
+            q, kc, vc = rows(qseed, NQ * D), rows(kseed, per_seq), rows(vseed, per_seq)
+            sinks = sdev.f32_normal(_seed(wl["dec_cfg"], layer, synth.TENSOR_SINKS), (NQ,),
+                                    "cpu").double().numpy()
+            self.dec.append(dict(
+                layer=layer, window=window,
+                q=q.reshape(self.n_seqs, NQ, D), kc=kc.reshape(self.n_seqs, DL, NKV, D),
+                vc=vc.reshape(self.n_seqs, DL, NKV, D), sinks=sinks))
+        self.q_seeds = [_seed(wl["pre_cfg"], layer, synth.TENSOR_Q)
+                        for layer, _ in wl["pre_layers"]]
+
+    def sample(self, index: int, rows: int, seqs: int):
+        """Runs one sample; returns dict(prefill_flops, prefill_s, decode_bytes, decode_s)."""
+        import torch
+
+        import oracle
+        from synth import device as sdev
+        oracle._load()
+        B, S = self.wl["B"], self.wl["S"]
+        pf = ps = 0.0
+        for p, qseed in zip(self.pre, self.q_seeds):
+            stride = S / rows
+            toks = ((np.arange(rows) + (index * 0.618034) % 1.0) * stride).astype(np.int64)
+            toks = np.clip(toks, 0, S - 1)
+            rws = [(int(i % B), int(t)) for i, t in enumerate(toks)]
+            q = torch.stack([sdev.bf16_normal_range(qseed, (b * S + t) * NQ * D, NQ * D, "cpu")
+                             for b, t in rws]).double().numpy().reshape(rows, NQ, D)
             t0 = time.perf_counter()
-            oracle.prefill_rows(q_rows, k, v, x["sinks"], x["pos"], window, rows)
-            dt = time.perf_counter() - t0
-            if dt >= per_layer / 3 or n >= PREFILL_S:
+            oracle.prefill_rows(q, p["k"], p["v"], p["sinks"], p["pos"], p["window"], rws)
+            ps += time.perf_counter() - t0
+            pf += sum(4.0 * D * NQ * (min(t + 1, p["window"]) if 0 < p["window"] < S else t + 1)
+                      for t in toks)
+        db = ds = 0.0
+        DL = self.wl["DL"]
+        for d in self.dec:
+            sel = [(index * seqs + j) % self.n_seqs for j in range(seqs)]
+            lens = np.full(seqs, DL, dtype=np.int64)
+            t0 = time.perf_counter()
+            oracle.decode(d["q"][sel], d["kc"][sel], d["vc"][sel], d["sinks"], lens, d["window"])
+            ds += time.perf_counter() - t0
+            db += decode_bytes(seqs, DL, d["window"])
+        return dict(prefill_flops=pf, prefill_s=ps, decode_bytes=db, decode_s=ds)
+
+    def calibrate(self, target_s: float):
+        """Rows per prefill layer and sequences per decode layer for a sample of
+        about target_s seconds."""
+        rows, seqs = 8, 1
+        while True:
+            r = self.sample(0, rows, seqs)
+            t = r["prefill_s"] + r["decode_s"]
+            if t >= target_s / 4 or rows >= 4096:
                 break
-            n = min(PREFILL_S, n * 4)
-        flops = sum(4.0 * D * NQ * (min(t + 1, window) if window > 0 else t + 1) for t in toks)
-        total_flops += flops
-        total_s += dt
-        nrows += n
-    return total_flops / total_s / 1e12, total_s, nrows, total_flops
+            rows *= 4
+        rows = max(8, min(4096, int(rows * target_s / max(t, 1e-3))))
+        return rows, seqs
 
 
-def run_reference(args, rank: int):
+def run_reference(args, rank: int, wl: dict):
+    """The reference arm: the fp64 oracle on the host cores, one bounded sample
+    of the workload per step (rank 0 only; other ranks exit without work)."""
     if rank != 0:
         return 0
-    value, secs, nrows, flops = oracle_sample()
+    sampler = OracleSampler(wl)
+    rows, seqs = sampler.calibrate(target_s=2.0)
+    for w in range(args.warmup):
+        sampler.sample(1000 + w, rows, seqs)
+    res = []
+    t_wall = time.perf_counter()
+    for s in range(args.steps):
+        res.append(sampler.sample(s, rows, seqs))
+    t_wall = time.perf_counter() - t_wall
+    pf = sum(r["prefill_flops"] for r in res)
+    ps = sum(r["prefill_s"] for r in res)
+    db = sum(r["decode_bytes"] for r in res)
+    dsec = sum(r["decode_s"] for r in res)
+    value = pf / ps / 1e12
     cores = host_cores()
+    sample = ("per step: %d evenly spaced query rows (all 64 heads) of each of the %d prefill "
+              "layers and %d sequence(s) of each of the %d decode layers; %.3g unmasked FLOPs and "
+              "%.3g decode bytes per step on average" % (
+                  rows, len(wl["pre_layers"]), seqs, len(wl["dec_layers"]), pf / args.steps,
+                  db / args.steps))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": secs * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "parallelism": "host cores"},
+        "ms_per_step": t_wall * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic: seeded recipe (synth), same "
+        "as the GPU arm", "config": step_config(wl),
+        "sample": sample,
+        "extrapolated": {"full_step_s": sum(prefill_flops(wl["B"], wl["S"], w)
+                                            for _, w in wl["pre_layers"]) * ps / pf +
+                         sum(decode_bytes(wl["DB"], wl["DL"], w)
+                             for _, w in wl["dec_layers"]) * dsec / db,
+                         "how": "one whole step at the sampled rates (prefill by unmasked FLOPs, "
+                                "decode by bytes); an extrapolation, not a measurement"},
+        "decode": {"value": db / dsec / 1e9, "unit": "GB/s"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": "%d evenly spaced query rows (all 64 heads) of the two prefill "
-                                   "layers, %.3g unmasked FLOPs" % (nrows, flops)},
+                         "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -215,12 +340,41 @@ def run_reference(args, rank: int):
 
 # ------------------------------------------------------------------ GPU leg
 
-def run_ours(args, rank: int, world: int):
+def _prefill_layer(cfg, layer, window, B, S, dev, gqa):
+    import torch
+
+    import synth
+    from synth import device as sdev
+    return dict(
+        q=sdev.bf16_normal(_seed(cfg, layer, synth.TENSOR_Q), (B, S, NQ, D), dev),
+        k=sdev.bf16_normal(_seed(cfg, layer, synth.TENSOR_K), (B, S, NKV, D), dev),
+        v=sdev.bf16_normal(_seed(cfg, layer, synth.TENSOR_V), (B, S, NKV, D), dev),
+        sinks=sdev.f32_normal(_seed(cfg, layer, synth.TENSOR_SINKS), (NQ,), dev),
+        pos=torch.arange(S, dtype=torch.int32, device=dev).repeat(B, 1).contiguous(),
+        window=window, out=torch.empty(B, S, NQ, D, dtype=torch.bfloat16, device=dev),
+        ws=torch.empty(gqa.prefill_workspace_bytes(B, S), dtype=torch.uint8, device=dev))
+
+
+def _decode_layer(cfg, layer, window, B, L, dev, gqa):
+    import torch
+
+    import synth
+    from synth import device as sdev
+    return dict(
+        q=sdev.bf16_normal(_seed(cfg, layer, synth.TENSOR_Q), (B, NQ, D), dev),
+        kc=sdev.bf16_normal(_seed(cfg, layer, synth.TENSOR_K), (B, L, NKV, D), dev),
+        vc=sdev.bf16_normal(_seed(cfg, layer, synth.TENSOR_V), (B, L, NKV, D), dev),
+        sinks=sdev.f32_normal(_seed(cfg, layer, synth.TENSOR_SINKS), (NQ,), dev),
+        len=torch.full((B,), L, dtype=torch.int32, device=dev), window=window,
+        ws=torch.empty(gqa.decode_workspace_bytes(B, L, window), dtype=torch.uint8, device=dev),
+        out=torch.empty(B, NQ, D, dtype=torch.bfloat16, device=dev))
+
+
+def run_ours(args, rank: int, world: int, wl: dict):
     import torch
     import torch.distributed as dist
 
     import attention_gqa_b200 as gqa
-    import synth
     from attention_gqa_b200 import shard
 
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -234,30 +388,12 @@ def run_ours(args, rank: int, world: int):
         dist.barrier()
     gqa.init()
     stream = torch.cuda.current_stream()
-
-    def to_dev(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    B, S, DB, DL = wl["B"], wl["S"], wl["DB"], wl["DL"]
+    pre_layers, dec_layers = wl["pre_layers"], wl["dec_layers"]
 
     # inputs resident in HBM
-    pre = []
-    for layer, window in PREFILL_LAYERS:
-        x = synth.make_prefill_inputs(2, layer, PREFILL_B, PREFILL_S)
-        pre.append(dict(q=to_dev(x["q"]), k=to_dev(x["k"]), v=to_dev(x["v"]),
-                        sinks=torch.from_numpy(x["sinks"]).to(dev),
-                        pos=torch.from_numpy(x["pos"]).to(dev), window=window,
-                        out=torch.empty(PREFILL_B, PREFILL_S, NQ, D, dtype=torch.bfloat16,
-                                        device=dev),
-                        ws=torch.empty(gqa.prefill_workspace_bytes(PREFILL_B, PREFILL_S),
-                                       dtype=torch.uint8, device=dev), host=x))
-    dec = []
-    for layer, window in DECODE_LAYERS:
-        x = synth.make_decode_inputs(4, layer, DECODE_B, DECODE_L)
-        ws = torch.empty(gqa.decode_workspace_bytes(DECODE_B, DECODE_L, window),
-                         dtype=torch.uint8, device=dev)
-        dec.append(dict(q=to_dev(x["q"]), kc=to_dev(x["kcache"]), vc=to_dev(x["vcache"]),
-                        sinks=torch.from_numpy(x["sinks"]).to(dev),
-                        len=torch.from_numpy(x["len"]).to(dev), window=window, ws=ws,
-                        out=torch.empty(DECODE_B, NQ, D, dtype=torch.bfloat16, device=dev)))
+    pre = [_prefill_layer(wl["pre_cfg"], layer, w, B, S, dev, gqa) for layer, w in pre_layers]
+    dec = [_decode_layer(wl["dec_cfg"], layer, w, DB, DL, dev, gqa) for layer, w in dec_layers]
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
     def step(ev=None):
@@ -277,7 +413,7 @@ def run_ours(args, rank: int, world: int):
             if ev is not None:
                 ev[i].record(stream)
 
-    n_marks = 1 + len(PREFILL_LAYERS) + len(DECODE_LAYERS)
+    n_marks = 1 + len(pre_layers) + len(dec_layers)
     for _ in range(args.warmup):
         flush.fill_(1)
         step()
@@ -303,42 +439,42 @@ def run_ours(args, rank: int, world: int):
                     for s in range(args.steps)])  # ms, [steps, kernels]
     seg_total = seg.sum(axis=0)                                       # ms per segment over K steps
     seg_total = np.array(shard.max_over_ranks(seg_total, dev))  # the slowest rank sets the time
-    npre = len(PREFILL_LAYERS)
+    npre = len(pre_layers)
     pre_ms = float(seg_total[:npre].sum()) / args.steps
     dec_ms = float(seg_total[npre:].sum()) / args.steps
     step_ms = pre_ms + dec_ms
-    pre_flops = sum(prefill_flops(PREFILL_B, PREFILL_S, w) for _, w in PREFILL_LAYERS)
-    dec_bytes = sum(decode_bytes(DECODE_B, DECODE_L, w) for _, w in DECODE_LAYERS)
+    pre_flops = sum(prefill_flops(B, S, w) for _, w in pre_layers)
+    dec_bytes = sum(decode_bytes(DB, DL, w) for _, w in dec_layers)
     value = world * pre_flops / (pre_ms * 1e-3) / 1e12
     dec_gbs = world * dec_bytes / (dec_ms * 1e-3) / 1e9
 
     hbm, tf_burst, tf_sus, peak_src = load_peaks()
+    peak = tf_sus if wl["peak"] == "sustained" else tf_burst
     # dominant kernel: the full-causal prefill layer
-    full_idx = [i for i, (_, w) in enumerate(PREFILL_LAYERS) if w <= 0][0]
+    full_idx = [i for i, (_, w) in enumerate(pre_layers) if w <= 0][0]
     full_ms = float(seg_total[full_idx]) / args.steps
-    full_tf = prefill_flops(PREFILL_B, PREFILL_S, 0) / (full_ms * 1e-3) / 1e12
-    dfull_idx = npre + [i for i, (_, w) in enumerate(DECODE_LAYERS) if w <= 0][0]
+    full_tf = prefill_flops(B, S, 0) / (full_ms * 1e-3) / 1e12
+    slid_idx = [i for i, (_, w) in enumerate(pre_layers) if w > 0][0]
+    slid_ms = float(seg_total[slid_idx]) / args.steps
+    slid_bytes = prefill_bytes(B, S)
+    dfull_idx = npre + [i for i, (_, w) in enumerate(dec_layers) if w <= 0][0]
     dfull_ms = float(seg_total[dfull_idx]) / args.steps
-    dfull_gbs = decode_bytes(DECODE_B, DECODE_L, 0) / (dfull_ms * 1e-3) / 1e9
+    dfull_gbs = decode_bytes(DB, DL, 0) / (dfull_ms * 1e-3) / 1e9
 
-    # end to end through the public API from pinned host buffers (prefill layers)
-    def pinned(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
-            torch.bfloat16).pin_memory()
+    # end to end through the public API from pinned host buffers (prefill layers):
+    # every step copies each layer's inputs in and its output out
     hostin = []
     h2d = d2h = 0
     for p in pre:
-        x = p["host"]
-        hq, hk, hv = pinned(x["q"]), pinned(x["k"]), pinned(x["v"])
-        hs, hp = torch.from_numpy(x["sinks"]).pin_memory(), torch.from_numpy(x["pos"]).pin_memory()
+        hq, hk, hv = (p[n].cpu().pin_memory() for n in ("q", "k", "v"))
+        hs, hp = p["sinks"].cpu().pin_memory(), p["pos"].cpu().pin_memory()
         ho = torch.empty(p["out"].shape, dtype=torch.bfloat16).pin_memory()
         hostin.append((hq, hk, hv, hs, hp, p["window"], ho))
         h2d += sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs, hp))
         d2h += ho.numel() * ho.element_size()
-    e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        for hq, hk, hv, hs, hp, w, ho in hostin:
-            gqa.prefill(hq, hk, hv, hs, hp, w, out=ho)
+    e2e_steps = max(3, min(args.steps, 20 if S <= 16384 else 3))
+    for hq, hk, hv, hs, hp, w, ho in hostin:
+        gqa.prefill(hq, hk, hv, hs, hp, w, out=ho)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     e0.record(stream)
@@ -350,31 +486,48 @@ def run_ours(args, rank: int, world: int):
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     e2e_ms = shard.max_over_ranks([e2e_ms], dev)[0]
     e2e_value = world * pre_flops / (e2e_ms * 1e-3) / 1e12
+    del hostin
 
     if rank == 0:
         cpu = None
         if world == 1:
-            v, secs, nrows, flops = oracle_sample()
-            cpu = {"value": v, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
-                   "sample": "%d evenly spaced query rows (all 64 heads) of the two prefill "
-                             "layers, %.3g unmasked FLOPs, %.1f s" % (nrows, flops, secs)}
-        traffic = profiled_traffic()
+            sampler = OracleSampler(wl, tensors={"pre": pre})
+            rows, seqs = sampler.calibrate(target_s=3.0)
+            res = [sampler.sample(i, rows, seqs) for i in range(4)]
+            pf = sum(r["prefill_flops"] for r in res)
+            ps = sum(r["prefill_s"] for r in res)
+            cpu = {"value": pf / ps / 1e12, "unit": "TFLOP/s", "cores": host_cores(),
+                   "kind": "oracle",
+                   "sample": "4 samples of %d evenly spaced query rows (all 64 heads) of each "
+                             "prefill layer: %.3g unmasked FLOPs in %.1f s" % (rows, pf, ps)}
+        traffic = profiled_traffic(os.path.join(
+            ROOT, "profiles", "prefill_kernel_full_S%d_traffic.txt" % S))
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic: seeded N(0,1) bf16 q/k/v and caches, N(0,1) fp32 sinks",
-            "config": {"workload": WORKLOAD, "l2": "flushed before every step (256 MB write)",
-                       "parallelism": "dp%d (independent replicas)" % world,
-                       "prefill_ms_per_step": pre_ms, "decode_ms_per_step": dec_ms,
+            "data": "synthetic: seeded N(0,1) bf16 q/k/v and caches, N(0,1) fp32 sinks "
+                    "(synth recipe, drawn on the device)",
+            "config": step_config(wl),
+            "parallelism": "dp%d (independent replicas)" % world,
+            "timing": {"prefill_ms_per_step": pre_ms, "decode_ms_per_step": dec_ms,
+                       "full_layer_ms": full_ms, "sliding_layer_ms": slid_ms,
                        "wall_s": t_wall},
             "roofline": {"kernel": "prefill (key rotation + prefill_kernel, full-causal layer, "
-                                   "S=4096)", "bound": "tensor",
-                         "achieved": full_tf, "peak": tf_burst, "unit": "TFLOP/s",
-                         "frac": full_tf / tf_burst, "peak_source": peak_src + " (burst)",
+                                   "B=%d S=%d)" % (B, S), "bound": "tensor",
+                         "achieved": full_tf, "peak": peak, "unit": "TFLOP/s",
+                         "frac": full_tf / peak,
+                         "peak_source": "%s (%s)" % (peak_src, wl["peak"]),
                          "traffic": traffic,
-                         "algorithmic_bytes": prefill_bytes(PREFILL_B, PREFILL_S),
+                         "algorithmic_bytes": prefill_bytes(B, S),
+                         "flops_per_launch": prefill_flops(B, S, 0),
                          "launch_ms": full_ms},
+            "sliding_roofline": {"kernel": "prefill (key rotation + prefill_band_kernel, W=128)",
+                                 "bound": "hbm",
+                                 "achieved": slid_bytes / (slid_ms * 1e-3) / 1e9, "peak": hbm,
+                                 "unit": "GB/s",
+                                 "frac": slid_bytes / (slid_ms * 1e-3) / 1e9 / hbm,
+                                 "algorithmic_bytes": slid_bytes, "launch_ms": slid_ms},
             "decode": {"value": dec_gbs, "unit": "GB/s", "frac": dec_gbs / world / hbm,
                        "peak": hbm, "full_layer_gbs": dfull_gbs,
                        "full_layer_frac": dfull_gbs / hbm, "full_layer_ms": dfull_ms},
@@ -383,9 +536,8 @@ def run_ours(args, rank: int, world: int):
                     "d2h_bytes_per_step": d2h, "what": "prefill layers via host buffers"},
             # per step: key rotation + attention per prefill layer; per decode layer the
             # split kernel, plus the combine kernel unless one split covers the range
-            "gpu_launches": args.steps * (2 * len(PREFILL_LAYERS) + sum(
-                1 if (min(w, DECODE_L) if w > 0 else DECODE_L) <= 256 else 2
-                for _, w in DECODE_LAYERS)),
+            "gpu_launches": args.steps * (2 * len(pre_layers) + sum(
+                1 if (min(w, DL) if w > 0 else DL) <= 256 else 2 for _, w in dec_layers)),
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -458,18 +610,7 @@ def run_long(args, name: str):
     torch.cuda.set_device(dev)
     gqa.init()
     stream = torch.cuda.current_stream()
-    bufs = []
-    for layer, window in layers:
-        def draw(shape, tid):
-            g = torch.Generator(device=dev)
-            g.manual_seed(0x6A77 ^ (cfg << 24) ^ (layer << 12) ^ tid)
-            return torch.randn(shape, generator=g, device=dev, dtype=torch.float32)
-        bufs.append(dict(
-            q=draw((B, S, NQ, D), 1).to(torch.bfloat16), k=draw((B, S, NKV, D), 2).to(torch.bfloat16),
-            v=draw((B, S, NKV, D), 3).to(torch.bfloat16), sinks=draw((NQ,), 4),
-            pos=torch.arange(S, dtype=torch.int32, device=dev).repeat(B, 1).contiguous(),
-            window=window, out=torch.empty(B, S, NQ, D, dtype=torch.bfloat16, device=dev),
-            ws=torch.empty(gqa.prefill_workspace_bytes(B, S), dtype=torch.uint8, device=dev)))
+    bufs = [_prefill_layer(cfg, layer, window, B, S, dev, gqa) for layer, window in layers]
     steps = max(1, min(args.steps, 20))
 
     def step(ev=None):
@@ -532,8 +673,8 @@ def run_long(args, name: str):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic: N(0,1) bf16 q/k/v and fp32 sinks drawn on the device (torch "
-                "generator seeded per layer), pos = token index",
+        "data": "synthetic: seeded N(0,1) bf16 q/k/v and fp32 sinks (synth recipe, drawn on "
+                "the device), pos = token index",
         "config": {"workload": desc,
                    "l2": "flushed before every step (256 MB write)" +
                          ("; every layer's inputs exceed L2" if prefill_bytes(B, S) > 126e6
@@ -709,29 +850,31 @@ def oracle_chunk_sample(p, start: int, n: int, budget_s: float = 6.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["step", "chunk16k"] + sorted(LONG_WORKLOADS),
-                    default="step",
-                    help="step: the default prefill + decode step; tiny256 / batch16k / "
-                         "seq128k / layers36: other prefill workloads; chunk16k: chunked "
-                         "prefill against a cache (one GPU, at most 20 timed steps)")
+    ap.add_argument("--workload", choices=sorted(STEP_WORKLOADS) + ["chunk16k"] +
+                    sorted(LONG_WORKLOADS), default="default",
+                    help="default: prefill B=1 S=131072 + decode B=64 L=8192; s4096: the same "
+                         "step with a B=1 S=4096 prefill; tiny256 / batch16k / seq128k / "
+                         "layers36: prefill-only workloads; chunk16k: chunked prefill against a "
+                         "cache (one GPU, at most 20 timed steps)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
-        return run_reference(args, rank)
-    if args.workload != "step":
-        if world > 1:
-            print("--workload %s runs on one GPU" % args.workload, file=sys.stderr)
-            return 2
-        if args.workload == "chunk16k":
-            return run_chunk(args)
-        return run_long(args, args.workload)
-    return run_ours(args, rank, world)
+        wl = STEP_WORKLOADS.get(args.workload, STEP_WORKLOADS["default"])
+        return run_reference(args, rank, wl)
+    if args.workload in STEP_WORKLOADS:
+        return run_ours(args, rank, world, STEP_WORKLOADS[args.workload])
+    if world > 1:
+        print("--workload %s runs on one GPU" % args.workload, file=sys.stderr)
+        return 2
+    if args.workload == "chunk16k":
+        return run_chunk(args)
+    return run_long(args, args.workload)
 
 
 if __name__ == "__main__":

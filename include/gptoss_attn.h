@@ -95,6 +95,27 @@ int gptoss_attn_init(void);
 int gptoss_attn_rope_table(const void** table);
 
 /*
+ * YaRN rotary scaling (techniques map row "YaRN RoPE scaling": rope_type yarn,
+ * factor 32; initial_context_length 4096 in the llm-atlas field tables). The
+ * pages leave the betas, the ramp and the attention factor out; this library
+ * uses the transformers yarn initialisation the row names, with beta_fast 32,
+ * beta_slow 1 and no truncation: pair k's frequency theta^(-2k/64) is blended
+ * with theta^(-2k/64) / 32 by a weight linear in k, 0 up to the pair whose
+ * wavelength fits 32 times into 4096 tokens (k ~ 8.09) and 1 from the pair
+ * where it fits once (k ~ 17.40); cos and sin are scaled by the attention
+ * factor 0.1 ln 32 + 1 (YaRN paper, Peng et al. 2023), so rotated queries and
+ * keys both carry it and the logits grow by its square.
+ *
+ * gptoss_attn_init_yarn() builds the current device's YaRN table (another
+ * 33.5 MB, same layout and evaluation as the plain one; allocates, call it
+ * before capturing work that uses the _yarn entry points); the _yarn entry
+ * points build it on first use. gptoss_attn_rope_table_yarn() returns its
+ * address like gptoss_attn_rope_table().
+ */
+int gptoss_attn_init_yarn(void);
+int gptoss_attn_rope_table_yarn(const void** table);
+
+/*
  * Bytes of device workspace gptoss_attn_prefill() needs: room for the rotated
  * keys, batch * seqlen * 8 * 64 bf16 values. Returns 0 for invalid sizes.
  */
@@ -124,6 +145,61 @@ int gptoss_attn_prefill(const void* q, const void* k, const void* v, const float
                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * gptoss_attn_prefill() that also stores, for every query row, the natural
+ * log of its softmax normaliser, sink included:
+ *   lse[b][i][h] = ln(exp(sigma_h) + sum_j exp(s_j))   fp32 [batch][seqlen][64]
+ * (4-byte aligned, caller-owned device memory). The backward pass
+ * (gptoss_attn_prefill_backward) takes it instead of recomputing it.
+ */
+int gptoss_attn_prefill_lse(const void* q, const void* k, const void* v, const float* sinks,
+                            const int32_t* pos, int window, void* out, float* lse, int batch,
+                            int seqlen, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream);
+
+/*
+ * Bytes of device workspace gptoss_attn_prefill_backward() needs: the rotated
+ * queries and keys (bf16) and two fp32 values per query row, plus alignment.
+ * Returns 0 for invalid sizes.
+ */
+size_t gptoss_attn_prefill_backward_workspace_bytes(int batch, int seqlen);
+
+/*
+ * Backward pass of gptoss_attn_prefill() (plain RoPE): given the upstream
+ * gradient dout of out, the gradients of L = sum(dout * out) with respect to
+ * q, k, v (the un-rotated inputs) and the sink logits. The pages print no
+ * backward; these are the derivatives of the forward defined above (the sink
+ * row of the techniques map makes the sink a softmax column with no value):
+ *   D_i = dout_i . out_i,  dS_ij = p_ij (dout_i . v_j - D_i)
+ *   dv_j = sum_i p_ij dout_i (over the 8 query heads of the group too)
+ *   dq_i = R(pos_i)^T sum_j dS_ij R(pos_j) k_j / 8
+ *   dk_j = R(pos_j)^T sum_i dS_ij R(pos_i) q_i / 8
+ *   dsinks[h] = -sum_{b,i} exp(sigma_h - lse_i) D_i
+ *   q, k, v, sinks, pos, window: the forward's inputs
+ *   out    bf16 [batch][seqlen][64][64], the forward's output
+ *   lse    fp32 [batch][seqlen][64], from gptoss_attn_prefill_lse()
+ *   dout   bf16 [batch][seqlen][64][64]
+ *   dq     bf16 [batch][seqlen][64][64];  dk, dv  bf16 [batch][seqlen][8][64]
+ *   dsinks fp32 [64] (overwritten; accumulated with atomics, so the order of
+ *          the fp32 additions varies from run to run)
+ *   workspace of gptoss_attn_prefill_backward_workspace_bytes() bytes.
+ * Products run on the tensor cores in bf16 with fp32 accumulation: the
+ * rotated q, k and the probabilities and dS are rounded to bf16 first. All
+ * gradients are written whole (no accumulation into the caller's buffers).
+ * Kernels on `stream`: the q and k rotations, a per-row preparation (D, the
+ * sink gradient), the dq kernel, the dk/dv kernel.
+ */
+int gptoss_attn_prefill_backward(const void* q, const void* k, const void* v, const float* sinks,
+                                 const int32_t* pos, int window, const void* out, const float* lse,
+                                 const void* dout, void* dq, void* dk, void* dv, float* dsinks,
+                                 int batch, int seqlen, void* workspace, size_t workspace_bytes,
+                                 cudaStream_t stream);
+
+/* gptoss_attn_prefill() with the YaRN rotation (see gptoss_attn_init_yarn). */
+int gptoss_attn_prefill_yarn(const void* q, const void* k, const void* v, const float* sinks,
+                             const int32_t* pos, int window, void* out, int batch, int seqlen,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Chunked prefill: the next n tokens of sequences whose first `start` tokens
  * are already in a key/value cache (a prompt prefilled in pieces, or several
  * new tokens at once against a cache). The same operation as
@@ -149,6 +225,13 @@ int gptoss_attn_prefill_chunk(const void* q, const void* k, const void* v, const
                               const int32_t* pos, int window, void* out, void* kcache,
                               void* vcache, int batch, int start, int n, int max_len,
                               cudaStream_t stream);
+
+/* gptoss_attn_prefill_chunk() with the YaRN rotation: the cached keys must have
+ * been rotated by YaRN too (by this call or gptoss_attn_prefill_yarn's layout). */
+int gptoss_attn_prefill_chunk_yarn(const void* q, const void* k, const void* v,
+                                   const float* sinks, const int32_t* pos, int window, void* out,
+                                   void* kcache, void* vcache, int batch, int start, int n,
+                                   int max_len, cudaStream_t stream);
 
 /*
  * Bytes of device workspace gptoss_attn_decode() needs for these sizes.
@@ -176,6 +259,14 @@ size_t gptoss_attn_decode_workspace_bytes(int batch, int max_len, int window);
 int gptoss_attn_decode(const void* q, const void* kcache, const void* vcache, const float* sinks,
                        const int32_t* len, int window, void* out, int batch, int max_len,
                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* gptoss_attn_decode() with the query rotated by YaRN at position len[b]-1;
+ * the cache must hold YaRN-rotated keys. max_len <= 131072 (the table's
+ * range), else GPTOSS_ATTN_ERR_BAD_SHAPE. Same workspace size. */
+int gptoss_attn_decode_yarn(const void* q, const void* kcache, const void* vcache,
+                            const float* sinks, const int32_t* len, int window, void* out,
+                            int batch, int max_len, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream);
 
 /*
  * Allocation-free decode. The gpt-oss pages have no counterpart: this entry

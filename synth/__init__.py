@@ -10,6 +10,7 @@ from .inputs import (  # noqa: F401
     f32_to_bf16_bits,
     bf16_bits_to_f64,
     bf16_normal,
+    bf16_normal_range,
     f32_normal,
     seed_for,
     TENSOR_Q,

@@ -103,6 +103,17 @@ def bf16_normal(seed: int, shape) -> np.ndarray:
     return out.reshape(shape)
 
 
+def bf16_normal_range(seed: int, start: int, count: int) -> np.ndarray:
+    """Elements ``start .. start+count-1`` (``start`` even) of ``bf16_normal(seed, ...)``
+    flattened: the generator is counter-based, so any slice is drawn on its own."""
+    assert start % 2 == 0
+    out = np.empty(count, dtype=np.uint16)
+    for s in range(0, count, _CHUNK):
+        c = min(_CHUNK, count - s)
+        out[s:s + c] = f32_to_bf16_bits(_normal_chunk(seed, start + s, c).astype(np.float32))
+    return out
+
+
 def f32_normal(seed: int, shape) -> np.ndarray:
     """N(0,1) samples rounded to fp32."""
     return normal(seed, int(np.prod(shape))).astype(np.float32).reshape(shape)
