@@ -823,6 +823,97 @@ def run_chunk(args):
     return 0
 
 
+BACKWARD_WORKLOADS = {
+    # name: (config id of the seed recipe, B, S, [(layer, window), ...], description)
+    "bwd4k": (2, 1, 4096, [(0, 128), (1, 0)],
+              "backward of the prefill B=1 S=4096 64q/8kv d64, one W=128 layer + one full-causal "
+              "layer (dq, dk, dv, dsinks from out, lse and a random dO)"),
+    "bwd16k": (3, 4, 16384, [(0, 128), (1, 0)],
+               "backward of the prefill B=4 S=16384 64q/8kv d64, one W=128 layer + one "
+               "full-causal layer"),
+}
+
+
+def run_backward(args, name: str):
+    """One GPU: a step is the backward pass of every layer of the workload once.
+    FLOPs follow the usual convention for attention backward: 2.5 times the
+    forward's unmasked FLOPs (the five products S, dP, dV, dK, dQ over the
+    visible pairs; the kernels recompute S and dP once more). Prints one line."""
+    import torch
+
+    import attention_gqa_b200 as gqa
+    import synth
+    from attention_gqa_b200 import build
+    from synth import device as sdev
+    build.build()
+    cfg, B, S, layers, desc = BACKWARD_WORKLOADS[name]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    gqa.init()
+    stream = torch.cuda.current_stream()
+    bufs = []
+    for layer, window in layers:
+        p = _prefill_layer(cfg, layer, window, B, S, dev, gqa)
+        p["out"], p["lse"] = gqa.prefill_lse(p["q"], p["k"], p["v"], p["sinks"], p["pos"], window)
+        p["dout"] = sdev.bf16_normal(_seed(cfg, layer, 5), (B, S, NQ, D), dev)
+        p["bws"] = torch.empty(gqa.prefill_backward_workspace_bytes(B, S), dtype=torch.uint8,
+                               device=dev)
+        bufs.append(p)
+    gqa.check()
+    steps = max(1, min(args.steps, 20))
+
+    def step(ev=None):
+        for i, p in enumerate(bufs):
+            if ev is not None:
+                ev[i].record(stream)
+            gqa.prefill_backward(p["q"], p["k"], p["v"], p["sinks"], p["pos"], p["window"],
+                                 p["out"], p["lse"], p["dout"], workspace=p["bws"])
+        if ev is not None:
+            ev[len(bufs)].record(stream)
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    gqa.check()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(bufs) + 1)]
+              for _ in range(steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        for s_ in range(steps):
+            flush.fill_(s_ & 0xFF)
+            step(events[s_])
+        torch.cuda.synchronize()
+    gqa.check()
+    seg = np.array([[events[s_][i].elapsed_time(events[s_][i + 1]) for i in range(len(bufs))]
+                    for s_ in range(steps)]).sum(axis=0) / steps
+    flops = [2.5 * prefill_flops(B, S, w) for _, w in layers]
+    step_ms = float(seg.sum())
+    value = sum(flops) / (step_ms * 1e-3) / 1e12
+    full = [i for i, (_, w) in enumerate(layers) if w <= 0][0]
+    full_tf = flops[full] / (seg[full] * 1e-3) / 1e12
+    hbm, tf_burst, tf_sus, peak_src = load_peaks()
+    line = {
+        "metric": "attention backward TFLOP/s (2.5x the unmasked forward FLOPs)", "value": value,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) bf16 q/k/v/dO and fp32 sinks (synth recipe, drawn on "
+                "the device), pos = token index",
+        "config": {"workload": desc, "l2": "flushed before every step (256 MB write)",
+                   "layer_ms": [float(x) for x in seg]},
+        "roofline": {"kernel": "backward (rotations + prep + bwd_dq_kernel + bwd_dkv_kernel), "
+                               "full-causal layer", "bound": "tensor", "achieved": full_tf,
+                     "peak": tf_burst, "unit": "TFLOP/s", "frac": full_tf / tf_burst,
+                     "peak_source": peak_src + " (burst)", "traffic": None,
+                     "launch_ms": float(seg[full])},
+        "gpu_launches": steps * 5 * len(layers),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def oracle_chunk_sample(p, start: int, n: int, budget_s: float = 6.0):
     """The fp64 oracle on evenly spaced query rows of a chunk (keys: the whole
     cached prefix plus the chunk); returns (TFLOP/s, s, rows, FLOPs)."""
@@ -854,11 +945,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(STEP_WORKLOADS) + ["chunk16k"] +
-                    sorted(LONG_WORKLOADS), default="default",
+                    sorted(LONG_WORKLOADS) + sorted(BACKWARD_WORKLOADS), default="default",
                     help="default: prefill B=1 S=131072 + decode B=64 L=8192; s4096: the same "
                          "step with a B=1 S=4096 prefill; tiny256 / batch16k / seq128k / "
                          "layers36: prefill-only workloads; chunk16k: chunked prefill against a "
-                         "cache (one GPU, at most 20 timed steps)")
+                         "cache; bwd4k / bwd16k: the backward pass (one GPU, at most 20 timed "
+                         "steps)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -874,6 +966,8 @@ def main():
         return 2
     if args.workload == "chunk16k":
         return run_chunk(args)
+    if args.workload in BACKWARD_WORKLOADS:
+        return run_backward(args, args.workload)
     return run_long(args, args.workload)
 
 

@@ -3,8 +3,10 @@ fp64 oracle's YaRN mode, through the C ABI.
 
 YaRN (techniques map row "YaRN RoPE scaling"; factor 32 over the 4096-token
 initial context of the llm-atlas field tables) changes only the rotary table:
-blended frequencies and cos/sin scaled by 0.1 ln 32 + 1. Same bars as the
-plain path: max-abs 2e-2 and mean-abs 2e-3 on the bf16 output.
+blended frequencies and cos/sin scaled by 0.1 ln 32 + 1. The bars are the plain
+path's (max-abs 2e-2, mean-abs 2e-3) scaled by the factor the logits grow by,
+(0.1 ln 32 + 1)^2 = 1.81: the output error comes from the bf16 rounding of the
+rotated q and k, which perturbs each logit in proportion to its size.
 """
 import math
 
@@ -15,12 +17,21 @@ import torch
 import attention_gqa_b200 as gqa
 import oracle
 import synth
-from tests._util import bits_to_dev, compare, dev_to_f64
+from tests import _util
+from tests._util import bits_to_dev, dev_to_f64
 
 pytestmark = pytest.mark.gpu
 
 NQ, NKV, D = 64, 8, 64
 MSCALE = 0.1 * math.log(32.0) + 1.0
+
+
+def compare(got, ref, what):
+    err = np.abs(got - ref)
+    assert np.all(np.isfinite(got)), what
+    assert err.max() <= _util.MAX_ABS_TOL * MSCALE ** 2, "%s: max abs err %.3e" % (what, err.max())
+    assert err.mean() <= _util.MEAN_ABS_TOL * MSCALE ** 2, "%s: mean abs err %.3e" % (
+        what, err.mean())
 
 
 def test_yarn_table_matches_oracle_rotation(cuda_device):
