@@ -177,6 +177,7 @@ static int prefill_impl(const void* q, const void* k, const void* v, const float
   args.sinks = sinks;
   args.rope = table_of(dev, rope);
   args.err = g_state[dev].err;
+  args.out = out;
   args.lse = lse;
   args.batch = batch;
   args.seqlen = seqlen;
@@ -238,6 +239,7 @@ static int prefill_chunk_impl(const void* q, const void* k, const void* v, const
   args.sinks = sinks;
   args.rope = table_of(dev, rope);
   args.err = g_state[dev].err;
+  args.out = out;
   args.lse = nullptr;
   args.batch = batch;
   args.seqlen = n;
@@ -427,10 +429,16 @@ int gptoss_attn_prefill_backward(const void* q, const void* k, const void* v, co
   const uint64_t kstr[3] = {kHeadDim * 2, kNumKvHeads * kHeadDim * 2,
                             S * kNumKvHeads * kHeadDim * 2};
   const uint32_t kbox[4] = {kHeadDim, 1, 128, 1};
-  if (!make_tmap_bf16_4d(&maps.q, ws + off[0], qdims, qstr, qbox) ||
-      !make_tmap_bf16_4d(&maps.dout, dout, qdims, qstr, qbox) ||
-      !make_tmap_bf16_4d(&maps.k, ws + off[1], kdims, kstr, kbox) ||
-      !make_tmap_bf16_4d(&maps.v, v, kdims, kstr, kbox))
+  const uint32_t qbox8[4] = {kHeadDim, kGroup, 8, 1};
+  const uint32_t kbox64[4] = {kHeadDim, 1, 64, 1};
+  if (!make_tmap_bf16_4d(&maps.q16, ws + off[0], qdims, qstr, qbox) ||
+      !make_tmap_bf16_4d(&maps.dout16, dout, qdims, qstr, qbox) ||
+      !make_tmap_bf16_4d(&maps.q8, ws + off[0], qdims, qstr, qbox8) ||
+      !make_tmap_bf16_4d(&maps.dout8, dout, qdims, qstr, qbox8) ||
+      !make_tmap_bf16_4d(&maps.k64, ws + off[1], kdims, kstr, kbox64) ||
+      !make_tmap_bf16_4d(&maps.v64, v, kdims, kstr, kbox64) ||
+      !make_tmap_bf16_4d(&maps.k128, ws + off[1], kdims, kstr, kbox) ||
+      !make_tmap_bf16_4d(&maps.v128, v, kdims, kstr, kbox))
     return GPTOSS_ATTN_ERR_TENSOR_MAP;
 
   BackwardArgs a;

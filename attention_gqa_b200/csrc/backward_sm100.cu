@@ -20,17 +20,20 @@
 //     so a 16-token tile of one group is 128 consecutive floats; the sink
 //     gradient (block sums, one atomic per head and block).
 //   bwd_dq_kernel: one CTA per (b, g, 16 tokens) = an M=128 tile of 16 tokens
-//     x 8 heads; over its key tiles: S = Q'K'^T and dP = dO V^T (tcgen05, fp32
-//     in TMEM), dS by the elementwise warpgroup (bf16 back into S's columns),
-//     dQ += dS K' (A from TMEM). dQ stays in TMEM until the item's end, is
-//     rotated back and stored as bf16.
+//     x 8 heads; over its 64-key tiles: S = Q'K'^T and dP = dO V^T (tcgen05,
+//     fp32 in TMEM), dS by the elementwise warpgroup (bf16 back into S's
+//     columns), dQ += dS K' (A from TMEM). dQ stays in TMEM until the item's
+//     end, is rotated back and stored as bf16.
 //   bwd_dkv_kernel: one CTA per (b, g, 128 keys) = M=128 keys; over the
-//     query tiles that see them: S^T = K'Q'^T, dP^T = V dO^T, P^T and dS^T by
-//     the elementwise warpgroup, dV += P^T dO and dK += dS^T Q' (A from TMEM,
-//     summing over the 8 heads of the group because they are rows of the
-//     tile). No atomics on dq, dk or dv.
-// Roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
-// warps 4-7 the elementwise warpgroup (thread = TMEM lane); warps 2-3 idle.
+//     8-token (64-row) query tiles that see them: S^T = K'Q'^T, dP^T = V dO^T,
+//     P^T and dS^T by the elementwise warpgroup, dV += P^T dO and dK += dS^T Q'
+//     (A from TMEM, summing over the 8 heads of the group because they are
+//     rows of the tile). No atomics on dq, dk or dv.
+// Each CTA takes 256 tensor-memory columns and ~100 KB of shared memory, so
+// two CTAs share an SM and one's elementwise work overlaps the other's MMAs.
+// Roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
+// warps 2-5 the elementwise warpgroup (thread = TMEM lane; warp w reads lanes
+// 32 (w % 4) .. 32 (w % 4) + 31).
 // Every pipeline wait is bounded like the forward kernels'.
 #include <cmath>
 
@@ -41,28 +44,31 @@ namespace gqa {
 namespace {
 namespace bwd {
 
-constexpr int kThreads = 256;
-constexpr int kTok = 16;      // query tokens per 128-row tile
-constexpr int kKeys = 128;    // keys per tile
+constexpr int kThreads = 192;
+constexpr int kTok = 16;      // query tokens per 128-row dQ tile
+constexpr int kKeys = 128;    // keys per dK/dV tile
+constexpr int kQKeys = 64;    // keys per step of the dQ kernel
+constexpr int kKTok = 8;      // query tokens (64 rows) per step of the dK/dV kernel
 constexpr int kStages = 2;
 constexpr uint32_t kTile = 128 * 128;  // 128 rows of 64 bf16
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kHalf = 64 * 128;   // 64 rows of 64 bf16
+constexpr uint32_t kTmemCols = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kScaleLog2 = 0.125f * kLog2e;
 constexpr float kScale = 0.125f;
-// TMEM columns: S (or S^T) [0,128), dP (dP^T) [128,256), dQ or dV [256,320), dK [320,384).
-constexpr uint32_t kColS = 0, kColP = 128, kColA = 256, kColB = 320;
+// TMEM columns: S (or S^T) [0,64), dP (dP^T) [64,128), dQ or dV [128,192), dK [192,256).
+constexpr uint32_t kColS = 0, kColP = 64, kColA = 128, kColB = 192;
 
 // dq kernel shared memory
 constexpr uint32_t kQOffQ = 0, kQOffDO = kTile, kQOffK = 2 * kTile;
-constexpr uint32_t kQOffV = kQOffK + kStages * kTile;
-constexpr uint32_t kQOffBar = kQOffV + kStages * kTile;
+constexpr uint32_t kQOffV = kQOffK + kStages * kHalf;
+constexpr uint32_t kQOffBar = kQOffV + kStages * kHalf;
 // dkv kernel shared memory
 constexpr uint32_t kKOffK = 0, kKOffV = kTile, kKOffQ = 2 * kTile;  // [stage]: Q', then dO
-constexpr uint32_t kKOffLD = kKOffQ + kStages * 2 * kTile;           // [stage]: lse2[128], D[128]
-constexpr uint32_t kKOffBar = kKOffLD + kStages * 1024;
-// one CTA per SM: the tensor memory allocation takes all 512 columns
-constexpr uint32_t kSmemBytes = 120 * 1024;
+constexpr uint32_t kKOffLD = kKOffQ + kStages * 2 * kHalf;           // [stage]: lse2[64], D[64]
+constexpr uint32_t kKOffBar = kKOffLD + kStages * 512;
+// two CTAs per SM (each takes half of the tensor memory)
+constexpr uint32_t kSmemBytes = 100 * 1024;
 static_assert(kQOffBar + 256 + 1024 <= kSmemBytes && kKOffBar + 256 + 1024 <= kSmemBytes, "smem");
 
 enum : int {
@@ -131,22 +137,23 @@ __device__ void teardown(uint32_t tmem) {
   }
 }
 
-// D = A B^T over head_dim 64 for two K-major 128-row tiles (4 MMAs, K = 16).
+// D = A B^T over head_dim 64 for a K-major 128-row tile A and a K-major
+// 64-row tile B (4 MMAs, K = 16): D is 128 x 64.
 __device__ __forceinline__ void mma_abt(uint32_t d_tmem, uint32_t a, uint32_t b) {
-  constexpr uint32_t idesc = idesc_bf16(128, 128, false);
+  constexpr uint32_t idesc = idesc_bf16(128, 64, false);
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk)
     mma_bf16_ss(d_tmem, sdesc_sw128(a + 32 * kk), sdesc_sw128(b + 32 * kk), idesc,
                 kk > 0 ? 1u : 0u);
 }
 
-// D (+)= A B with A bf16 [128 x 128] in TMEM and B a 128-row tile read
+// D (+)= A B with A bf16 [128 x 64] in TMEM and B a 64-row tile read
 // MN-major (rows = the contraction, 64 bf16 per row = the N columns).
 __device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint32_t b,
                                            bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16(128, kHeadDim, true);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
+  for (int kk = 0; kk < 4; ++kk)
     mma_bf16_ts(d_tmem, a_tmem + 8 * kk, sdesc_sw128(b + 2048 * kk), idesc,
                 (accumulate || kk > 0) ? 1u : 0u);
 }
@@ -218,7 +225,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BackwardArgs a) {
 }
 
 // dQ for one (b, g, 16-token) tile per CTA.
-__global__ void __launch_bounds__(bwd::kThreads, 1)
+__global__ void __launch_bounds__(bwd::kThreads, 2)
     bwd_dq_kernel(const __grid_constant__ BackwardMaps maps, const BackwardArgs a) {
   using namespace bwd;
   extern __shared__ uint8_t smem_raw[];
@@ -236,27 +243,27 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   const int g = (idx % per_tile) % kNumKvHeads, b = (idx % per_tile) / kNumKvHeads;
   const int q0 = qt * kTok;
   const int tlast = min(q0 + kTok - 1, S - 1);
-  const int jt0 = W > 0 ? max(0, q0 - W + 1) / kKeys : 0;
-  const int n_tiles = tlast / kKeys - jt0 + 1;
+  const int jt0 = W > 0 ? max(0, q0 - W + 1) / kQKeys : 0;
+  const int n_tiles = tlast / kQKeys - jt0 + 1;
 
   if (warp == 0) {
     if (lane == 0 && !skip) {
-      prefetch_tensormap(&maps.q);
-      prefetch_tensormap(&maps.dout);
-      prefetch_tensormap(&maps.k);
-      prefetch_tensormap(&maps.v);
+      prefetch_tensormap(&maps.q16);
+      prefetch_tensormap(&maps.dout16);
+      prefetch_tensormap(&maps.k64);
+      prefetch_tensormap(&maps.v64);
       mbar_arrive_expect_tx(ctx.bar(BAR_Q_FULL), 2 * kTile);
-      tma_load_4d(ctx.sbase + kQOffQ, &maps.q, ctx.bar(BAR_Q_FULL), 0, g * kGroup, q0, b);
-      tma_load_4d(ctx.sbase + kQOffDO, &maps.dout, ctx.bar(BAR_Q_FULL), 0, g * kGroup, q0, b);
+      tma_load_4d(ctx.sbase + kQOffQ, &maps.q16, ctx.bar(BAR_Q_FULL), 0, g * kGroup, q0, b);
+      tma_load_4d(ctx.sbase + kQOffDO, &maps.dout16, ctx.bar(BAR_Q_FULL), 0, g * kGroup, q0, b);
       int j = 0;
       for (; j < n_tiles; ++j) {
         const int s = j % kStages;
         if (j >= kStages && !ctx.wait(BAR_KV_EMPTY + s, ((j / kStages) - 1) & 1)) break;
-        mbar_arrive_expect_tx(ctx.bar(BAR_KV_FULL + s), 2 * kTile);
-        tma_load_4d(ctx.sbase + kQOffK + s * kTile, &maps.k, ctx.bar(BAR_KV_FULL + s), 0, g,
-                    (jt0 + j) * kKeys, b);
-        tma_load_4d(ctx.sbase + kQOffV + s * kTile, &maps.v, ctx.bar(BAR_KV_FULL + s), 0, g,
-                    (jt0 + j) * kKeys, b);
+        mbar_arrive_expect_tx(ctx.bar(BAR_KV_FULL + s), 2 * kHalf);
+        tma_load_4d(ctx.sbase + kQOffK + s * kHalf, &maps.k64, ctx.bar(BAR_KV_FULL + s), 0, g,
+                    (jt0 + j) * kQKeys, b);
+        tma_load_4d(ctx.sbase + kQOffV + s * kHalf, &maps.v64, ctx.bar(BAR_KV_FULL + s), 0, g,
+                    (jt0 + j) * kQKeys, b);
       }
       if (*ctx.abort_flag) {
         volatile int never = 0;
@@ -279,17 +286,17 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         tc_fence_after_sync();
         if (j > 0) {
           const int sp = (j - 1) % kStages;
-          mma_tmem_a(tmem + kColA, tmem + kColS, ctx.sbase + kQOffK + sp * kTile, j > 1);
+          mma_tmem_a(tmem + kColA, tmem + kColS, ctx.sbase + kQOffK + sp * kHalf, j > 1);
           mma_commit(ctx.bar(BAR_KV_EMPTY + sp));
         }
-        mma_abt(tmem + kColS, ctx.sbase + kQOffQ, ctx.sbase + kQOffK + s * kTile);
-        mma_abt(tmem + kColP, ctx.sbase + kQOffDO, ctx.sbase + kQOffV + s * kTile);
+        mma_abt(tmem + kColS, ctx.sbase + kQOffQ, ctx.sbase + kQOffK + s * kHalf);
+        mma_abt(tmem + kColP, ctx.sbase + kQOffDO, ctx.sbase + kQOffV + s * kHalf);
         mma_commit(ctx.bar(BAR_S_FULL));
       }
       if (ok && (ok = ctx.wait(BAR_E_DONE, (n_tiles - 1) & 1))) {
         tc_fence_after_sync();
         const int sp = (n_tiles - 1) % kStages;
-        mma_tmem_a(tmem + kColA, tmem + kColS, ctx.sbase + kQOffK + sp * kTile, n_tiles > 1);
+        mma_tmem_a(tmem + kColA, tmem + kColS, ctx.sbase + kQOffK + sp * kHalf, n_tiles > 1);
         mma_commit(ctx.bar(BAR_KV_EMPTY + sp));
         mma_commit(ctx.bar(BAR_ACC_FULL));
       }
@@ -297,7 +304,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       volatile int never = 0;
       mbar_wait(ctx.bar(BAR_MMA_DONE), 0, &never, nullptr, 0, kWaitTimeoutNs);
     }
-  } else if (warp >= 4) {
+  } else {
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // row: token q0 + r/8, head g*8 + r%8
     const int t = q0 + (r >> 3);
@@ -313,11 +320,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     for (int j = 0; ok && j < n_tiles; ++j) {
       if (!(ok = ctx.wait_warp(BAR_S_FULL, j & 1))) break;
       tc_fence_after_sync();
-      const int kb = (jt0 + j) * kKeys;
+      const int kb = (jt0 + j) * kQKeys;
       const int c_hi = t - kb;                           // visible columns [c_lo, c_hi]
       const int c_lo = W > 0 ? t - W + 1 - kb : -1;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t sv[32], pv[32], out[16];
         tmem_ld32(tmem + lane_off + kColS + 32 * c, sv);
         tmem_ld32(tmem + lane_off + kColP + 32 * c, pv);
@@ -358,7 +365,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 }
 
 // dK and dV for one (b, g, 128-key) tile per CTA.
-__global__ void __launch_bounds__(bwd::kThreads, 1)
+__global__ void __launch_bounds__(bwd::kThreads, 2)
     bwd_dkv_kernel(const __grid_constant__ BackwardMaps maps, const BackwardArgs a) {
   using namespace bwd;
   extern __shared__ uint8_t smem_raw[];
@@ -377,34 +384,34 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   const int kb = kt * kKeys;
   // query tokens that see a key of this tile: [kb, t_max]
   const int t_max = W > 0 ? min(S - 1, kb + kKeys - 1 + W - 1) : S - 1;
-  const int qt0 = kb / kTok;
-  const int n_tiles = t_max / kTok - qt0 + 1;
+  const int qt0 = kb / kKTok;
+  const int n_tiles = t_max / kKTok - qt0 + 1;
   const float* lse2_g = a.lse2 + (static_cast<int64_t>(b) * kNumKvHeads + g) * S * kGroup;
   const float* dd_g = a.dd + (static_cast<int64_t>(b) * kNumKvHeads + g) * S * kGroup;
 
   if (warp == 0) {
     if (lane == 0 && !skip) {
-      prefetch_tensormap(&maps.q);
-      prefetch_tensormap(&maps.dout);
-      prefetch_tensormap(&maps.k);
-      prefetch_tensormap(&maps.v);
+      prefetch_tensormap(&maps.q8);
+      prefetch_tensormap(&maps.dout8);
+      prefetch_tensormap(&maps.k128);
+      prefetch_tensormap(&maps.v128);
       mbar_arrive_expect_tx(ctx.bar(BAR_KV_FULL), 2 * kTile);
-      tma_load_4d(ctx.sbase + kKOffK, &maps.k, ctx.bar(BAR_KV_FULL), 0, g, kb, b);
-      tma_load_4d(ctx.sbase + kKOffV, &maps.v, ctx.bar(BAR_KV_FULL), 0, g, kb, b);
+      tma_load_4d(ctx.sbase + kKOffK, &maps.k128, ctx.bar(BAR_KV_FULL), 0, g, kb, b);
+      tma_load_4d(ctx.sbase + kKOffV, &maps.v128, ctx.bar(BAR_KV_FULL), 0, g, kb, b);
       int j = 0;
       for (; j < n_tiles; ++j) {
         const int s = j % kStages;
         if (j >= kStages && !ctx.wait(BAR_Q_EMPTY + s, ((j / kStages) - 1) & 1)) break;
-        const int t0 = (qt0 + j) * kTok;
-        const uint32_t st = ctx.sbase + kKOffQ + s * 2 * kTile;
-        const uint32_t ld = ctx.sbase + kKOffLD + s * 1024;
-        // lse2 and D of the tile's 128 rows: 512 contiguous bytes each (the
+        const int t0 = (qt0 + j) * kKTok;
+        const uint32_t st = ctx.sbase + kKOffQ + s * 2 * kHalf;
+        const uint32_t ld = ctx.sbase + kKOffLD + s * 512;
+        // lse2 and D of the step's 64 rows: 256 contiguous bytes each (the
         // arrays are padded by one tile, rows past the sequence are masked)
-        mbar_arrive_expect_tx(ctx.bar(BAR_Q_FULL + s), 2 * kTile + 1024);
-        tma_load_4d(st, &maps.q, ctx.bar(BAR_Q_FULL + s), 0, g * kGroup, t0, b);
-        tma_load_4d(st + kTile, &maps.dout, ctx.bar(BAR_Q_FULL + s), 0, g * kGroup, t0, b);
-        bulk_load(ld, lse2_g + static_cast<int64_t>(t0) * kGroup, 512, ctx.bar(BAR_Q_FULL + s));
-        bulk_load(ld + 512, dd_g + static_cast<int64_t>(t0) * kGroup, 512,
+        mbar_arrive_expect_tx(ctx.bar(BAR_Q_FULL + s), 2 * kHalf + 512);
+        tma_load_4d(st, &maps.q8, ctx.bar(BAR_Q_FULL + s), 0, g * kGroup, t0, b);
+        tma_load_4d(st + kHalf, &maps.dout8, ctx.bar(BAR_Q_FULL + s), 0, g * kGroup, t0, b);
+        bulk_load(ld, lse2_g + static_cast<int64_t>(t0) * kGroup, 256, ctx.bar(BAR_Q_FULL + s));
+        bulk_load(ld + 256, dd_g + static_cast<int64_t>(t0) * kGroup, 256,
                   ctx.bar(BAR_Q_FULL + s));
       }
       if (*ctx.abort_flag) {
@@ -425,21 +432,21 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         tc_fence_after_sync();
         if (j > 0) {
           const int sp = (j - 1) % kStages;
-          const uint32_t st = ctx.sbase + kKOffQ + sp * 2 * kTile;
-          mma_tmem_a(tmem + kColA, tmem + kColS, st + kTile, j > 1);  // dV += P^T dO
+          const uint32_t st = ctx.sbase + kKOffQ + sp * 2 * kHalf;
+          mma_tmem_a(tmem + kColA, tmem + kColS, st + kHalf, j > 1);  // dV += P^T dO
           mma_tmem_a(tmem + kColB, tmem + kColP, st, j > 1);          // dK += dS^T Q'
           mma_commit(ctx.bar(BAR_Q_EMPTY + sp));
         }
-        const uint32_t st = ctx.sbase + kKOffQ + s * 2 * kTile;
+        const uint32_t st = ctx.sbase + kKOffQ + s * 2 * kHalf;
         mma_abt(tmem + kColS, ctx.sbase + kKOffK, st);           // S^T = K' Q'^T
-        mma_abt(tmem + kColP, ctx.sbase + kKOffV, st + kTile);   // dP^T = V dO^T
+        mma_abt(tmem + kColP, ctx.sbase + kKOffV, st + kHalf);   // dP^T = V dO^T
         mma_commit(ctx.bar(BAR_S_FULL));
       }
       if (ok && (ok = ctx.wait(BAR_E_DONE, (n_tiles - 1) & 1))) {
         tc_fence_after_sync();
         const int sp = (n_tiles - 1) % kStages;
-        const uint32_t st = ctx.sbase + kKOffQ + sp * 2 * kTile;
-        mma_tmem_a(tmem + kColA, tmem + kColS, st + kTile, n_tiles > 1);
+        const uint32_t st = ctx.sbase + kKOffQ + sp * 2 * kHalf;
+        mma_tmem_a(tmem + kColA, tmem + kColS, st + kHalf, n_tiles > 1);
         mma_tmem_a(tmem + kColB, tmem + kColP, st, n_tiles > 1);
         mma_commit(ctx.bar(BAR_Q_EMPTY + sp));
         mma_commit(ctx.bar(BAR_ACC_FULL));
@@ -448,7 +455,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       volatile int never = 0;
       mbar_wait(ctx.bar(BAR_MMA_DONE), 0, &never, nullptr, 0, kWaitTimeoutNs);
     }
-  } else if (warp >= 4) {
+  } else {
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // key kb + r
     const int kj = kb + r;
@@ -458,13 +465,13 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       const int s = j % kStages;
       if (!(ok = ctx.wait_warp(BAR_S_FULL, j & 1))) break;
       tc_fence_after_sync();
-      const int t0 = (qt0 + j) * kTok;
-      const float* ld = reinterpret_cast<const float*>(smem + kKOffLD + s * 1024);
+      const int t0 = (qt0 + j) * kKTok;
+      const float* ld = reinterpret_cast<const float*>(smem + kKOffLD + s * 512);
       // column col is token t0 + col/8: visible iff kj <= t < S and t < kj + W
       const int lo_t = kj - t0;                              // first visible token offset
       const int hi_t = min(S - 1 - t0, W > 0 ? kj + W - 1 - t0 : 1 << 30);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t sv[32], pv[32], pw[16], dw[16];
         tmem_ld32(tmem + lane_off + kColS + 32 * c, sv);
         tmem_ld32(tmem + lane_off + kColP + 32 * c, pv);
@@ -477,7 +484,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
             const int tt = col >> 3;
             const bool vis = tt >= lo_t && tt <= hi_t;
             p[u] = vis ? ex2_approx(__uint_as_float(sv[e + u]) * kScaleLog2 - ld[col]) : 0.f;
-            ds[u] = p[u] * (__uint_as_float(pv[e + u]) - ld[128 + col]) * kScale;
+            ds[u] = p[u] * (__uint_as_float(pv[e + u]) - ld[64 + col]) * kScale;
           }
           pw[e / 2] = pack_bf16x2(p[0], p[1]);
           dw[e / 2] = pack_bf16x2(ds[0], ds[1]);

@@ -29,6 +29,7 @@ struct PrefillArgs {
   const float* sinks;   // [64]
   const float2* rope;   // [kMaxPosition][32] (cos, sin)
   int* err;             // device error word
+  void* out;            // [B][S][64][64] bf16, the output (also reached through maps.o)
   float* lse;           // [B][S][64] natural-log softmax normaliser per row (sink
                         // included), written when not null; indexed like out
   int batch;
@@ -114,8 +115,10 @@ struct BackwardArgs {
 };
 
 struct BackwardMaps {
-  CUtensorMap q, dout;     // rotated q and dO: boxes (64, 8, 16, 1)
-  CUtensorMap k, v;        // rotated k and v: boxes (64, 1, 128, 1)
+  CUtensorMap q16, dout16;  // rotated q and dO, boxes (64, 8, 16, 1): 128-row dQ tiles
+  CUtensorMap q8, dout8;    // the same, boxes (64, 8, 8, 1): 64-row steps of dK/dV
+  CUtensorMap k64, v64;     // rotated k and v, boxes (64, 1, 64, 1): steps of dQ
+  CUtensorMap k128, v128;   // the same, boxes (64, 1, 128, 1): dK/dV tiles
 };
 
 int backward_q_tiles(int seqlen);
