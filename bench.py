@@ -169,6 +169,21 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+EXP_PER_CLK_PER_SM = 16   # ex2.approx.ftz.f32 results per clock per SM on B200 (probe)
+NUM_SMS = 148
+
+
+def exp_roofline(flops: float, ms: float, clocks: dict) -> dict:
+    """Exponential-unit roofline of a full-causal prefill launch: FLOPs / 256 exps."""
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965
+    achieved = flops / 256.0 / (ms * 1e-3) / 1e9
+    peak = EXP_PER_CLK_PER_SM * NUM_SMS * mhz * 1e6 / 1e9
+    return {"bound": "alu (exponential unit)", "achieved": achieved, "peak": peak,
+            "unit": "Gexp/s", "frac": achieved / peak,
+            "peak_basis": "16 ex2 results/clk/SM (measured) x 148 SMs x %.0f MHz median SM clock"
+                          % mhz}
+
+
 def host_cores() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -522,6 +537,10 @@ def run_ours(args, rank: int, world: int, wl: dict):
                          "algorithmic_bytes": prefill_bytes(B, S),
                          "flops_per_launch": prefill_flops(B, S, 0),
                          "launch_ms": full_ms},
+            # the unit that binds prefill_kernel at head_dim 64: one exp2 per visible
+            # (query, key, head), 16 results per clock per SM (measured), 148 SMs, at the
+            # median SM clock seen during the timed steps
+            "exp_roofline": exp_roofline(prefill_flops(B, S, 0), full_ms, clk.summary()),
             "sliding_roofline": {"kernel": "prefill (key rotation + prefill_band_kernel, W=128)",
                                  "bound": "hbm",
                                  "achieved": slid_bytes / (slid_ms * 1e-3) / 1e9, "peak": hbm,
@@ -687,6 +706,7 @@ def run_long(args, name: str):
                      "frac": full_tf / tf_sus, "peak_source": peak_src + " (sustained)",
                      "traffic": None, "algorithmic_bytes": prefill_bytes(B, S),
                      "launch_ms": full_ms},
+        "exp_roofline": exp_roofline(prefill_flops(B, S, 0), full_ms, clk.summary()),
         "sliding_roofline": {"bound": "hbm", "achieved": slid_bytes / (slid_ms * 1e-3) / 1e9,
                              "peak": hbm, "unit": "GB/s",
                              "frac": slid_bytes / (slid_ms * 1e-3) / 1e9 / hbm},
@@ -938,19 +958,64 @@ def oracle_chunk_sample(p, start: int, n: int, budget_s: float = 6.0):
     return flops / dt / 1e12, dt, m, flops
 
 
+def run_call(args):
+    """One GPU, no timing: one attention operation run --reps times on seeded
+    inputs (the command the ncu captures under profiles/ run). --op fwd runs
+    the prefill, bwd the backward pass, dec the decode."""
+    import torch
+
+    import attention_gqa_b200 as gqa
+    from attention_gqa_b200 import build
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    gqa.init()
+    B, S, W = args.batch, args.seqlen, args.window
+    if args.op == "dec":
+        d = _decode_layer(4, 0, W, B, S, dev, gqa)
+        for _ in range(args.reps):
+            gqa.decode(d["q"], d["kc"], d["vc"], d["sinks"], d["len"], W, out=d["out"],
+                       workspace=d["ws"])
+    else:
+        p = _prefill_layer(9, 0, W, B, S, dev, gqa)
+        if args.op == "fwd":
+            for _ in range(args.reps):
+                gqa.prefill(p["q"], p["k"], p["v"], p["sinks"], p["pos"], W, out=p["out"],
+                            workspace=p["ws"])
+        else:
+            import synth
+            from synth import device as sdev
+            out, lse = gqa.prefill_lse(p["q"], p["k"], p["v"], p["sinks"], p["pos"], W)
+            dout = sdev.bf16_normal(synth.seed_for(9, 0, 5), (B, S, NQ, D), dev)
+            ws = torch.empty(gqa.prefill_backward_workspace_bytes(B, S), dtype=torch.uint8,
+                             device=dev)
+            for _ in range(args.reps):
+                gqa.prefill_backward(p["q"], p["k"], p["v"], p["sinks"], p["pos"], W, out, lse,
+                                     dout, workspace=ws)
+    gqa.check()
+    torch.cuda.synchronize()
+    print(json.dumps({"call": args.op, "batch": B, "seqlen": S, "window": W, "reps": args.reps}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(STEP_WORKLOADS) + ["chunk16k"] +
+    ap.add_argument("--workload", choices=sorted(STEP_WORKLOADS) + ["chunk16k", "call"] +
                     sorted(LONG_WORKLOADS) + sorted(BACKWARD_WORKLOADS), default="default",
                     help="default: prefill B=1 S=131072 + decode B=64 L=8192; s4096: the same "
                          "step with a B=1 S=4096 prefill; tiny256 / batch16k / seq128k / "
                          "layers36: prefill-only workloads; chunk16k: chunked prefill against a "
                          "cache; bwd4k / bwd16k: the backward pass (one GPU, at most 20 timed "
-                         "steps)")
+                         "steps); call: run --op once per --reps, untimed (for profilers)")
+    ap.add_argument("--op", choices=["fwd", "bwd", "dec"], default="fwd")
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--seqlen", type=int, default=16384)
+    ap.add_argument("--window", type=int, default=0)
+    ap.add_argument("--reps", type=int, default=2)
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -966,6 +1031,8 @@ def main():
         return 2
     if args.workload == "chunk16k":
         return run_chunk(args)
+    if args.workload == "call":
+        return run_call(args)
     if args.workload in BACKWARD_WORKLOADS:
         return run_backward(args, args.workload)
     return run_long(args, args.workload)
