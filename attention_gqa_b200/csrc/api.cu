@@ -187,6 +187,7 @@ static int prefill_impl(const void* q, const void* k, const void* v, const float
   args.n_qtiles = (seqlen + 31) / 32;
   args.n_items = prefill_items(batch, seqlen, args.window);
   args.grid = g_state[dev].num_sms;
+  args.order_chunk = prefill_order_chunk(batch, seqlen, args.grid);
   if (launch_rope_rows(k, pos, args.rope, workspace, batch, seqlen, seqlen, 0, kNumKvHeads,
                        args.grid * 8, args.err, stream) != cudaSuccess)
     return GPTOSS_ATTN_ERR_LAUNCH;
@@ -249,6 +250,7 @@ static int prefill_chunk_impl(const void* q, const void* k, const void* v, const
   args.n_qtiles = (n + 31) / 32;
   args.n_items = prefill_items(batch, n, args.window);
   args.grid = g_state[dev].num_sms;
+  args.order_chunk = prefill_order_chunk(batch, keys, args.grid);
   // values into the cache, then the rotated keys, then the attention (which
   // may start during the key rotation and waits for it before reading keys)
   const size_t row = static_cast<size_t>(kNumKvHeads) * kHeadDim * 2;

@@ -40,6 +40,9 @@ struct PrefillArgs {
   int n_qtiles;         // ceil(seqlen / 32)
   int n_items;          // work items (prefill_items)
   int grid;             // persistent CTAs (the device's SM count)
+  int order_chunk;      // 0: items by query tile (longest first), then group; C > 0:
+                        // chunks of C query tiles (longest first), inside a chunk by
+                        // (batch, group), so a wave reads few groups' keys and values
 };
 
 struct PrefillMaps {
@@ -51,6 +54,8 @@ struct PrefillMaps {
 bool prefill_uses_band(int window);
 // Work items of one prefill launch.
 int prefill_items(int batch, int seqlen, int window);
+// Item order of the full-causal kernel for these sizes (PrefillArgs::order_chunk).
+int prefill_order_chunk(int batch, int keys, int grid);
 
 // Launches the prefill kernel; returns a cudaError_t.
 cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream);

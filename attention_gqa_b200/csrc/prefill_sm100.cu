@@ -132,17 +132,33 @@ struct Item {
   int b, g, q0, jt0, n_tiles;
 };
 
-// The k-th item of CTA `cta` in snake order over items sorted longest first
-// (query tile descending, then kv head, then batch); false past the end.
+// The k-th item of CTA `cta` in snake order over items sorted longest first;
+// false past the end. Order 0: query tile descending, then kv head, then
+// batch. Order C > 0 (long sequences): chunks of C query tiles from the end,
+// inside a chunk (batch, kv head) outer and query tile descending inner, so
+// the CTAs of a wave stream the keys and values of only a few (b, g) pairs and
+// those stay in L2 (with every pair active at once they do not fit).
 __device__ __forceinline__ bool item_for(const PrefillArgs& a, int k, int cta, Item* it) {
   const int grid = static_cast<int>(gridDim.x);
   const int idx = (k & 1) ? (k + 1) * grid - 1 - cta : k * grid + cta;
   if (idx >= a.n_items) return false;
-  const int per_tile = kNumKvHeads * a.batch;
-  const int qt = a.n_qtiles - 1 - idx / per_tile;
-  const int rem = idx % per_tile;
-  it->g = rem % kNumKvHeads;
-  it->b = rem / kNumKvHeads;
+  const int n_bg = kNumKvHeads * a.batch;
+  int qt, bg;
+  if (a.order_chunk == 0) {
+    qt = a.n_qtiles - 1 - idx / n_bg;
+    bg = idx % n_bg;
+  } else {
+    const int C = a.order_chunk;
+    const int c = idx / (C * n_bg);
+    const int r = idx - c * C * n_bg;
+    const int top = a.n_qtiles - 1 - c * C;  // highest query tile of the chunk
+    const int cc = min(C, top + 1);          // query tiles in the chunk
+    bg = r / cc;
+    qt = top - r % cc;
+  }
+  // bg = b * 8 + g
+  it->g = bg % kNumKvHeads;
+  it->b = bg / kNumKvHeads;
   it->q0 = qt * kBlockQ;
   // key index of the item's first and last query token
   const int kq0 = a.q_start + it->q0;
@@ -1077,6 +1093,17 @@ bool prefill_uses_band(int window) { return window > 0 && window <= 128; }
 int prefill_items(int batch, int seqlen, int window) {
   const int tokens = prefill_uses_band(window) ? band::kTokens : kBlockQ;
   return (seqlen + tokens - 1) / tokens * kNumKvHeads * batch;
+}
+
+// While the keys and values of every (b, g) pair fit in half of L2 (126 MB),
+// the plain longest-first order balances best. Beyond that, chunks of C query
+// tiles with C large enough that the ~grid/C pairs a wave touches hold at most
+// 64 MB of keys and values (256 bytes per key and kv head).
+int prefill_order_chunk(int batch, int keys, int grid) {
+  const double kv_bytes = 256.0 * keys;  // one (b, g) pair
+  if (kv_bytes * kNumKvHeads * batch <= 64.0 * 1024 * 1024) return 0;
+  const int c = static_cast<int>(std::ceil(grid * kv_bytes / (64.0 * 1024 * 1024)));
+  return c < 1 ? 1 : c;
 }
 
 // Both attention kernels are launched with programmatic stream serialization:
