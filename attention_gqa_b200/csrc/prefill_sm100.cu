@@ -241,6 +241,45 @@ __device__ __forceinline__ uint32_t stage_rope_rows(const PrefillArgs& a, int b,
   return bytes;
 }
 
+// Rotary positions of tokens q0 .. q0+N-1 of sequence b (0 past the sequence
+// end). The loads are independent, so they cost one round trip to memory.
+template <int N>
+__device__ __forceinline__ void load_positions(const PrefillArgs& a, int b, int q0, int (&p)[N]) {
+#pragma unroll
+  for (int t = 0; t < N; ++t)
+    p[t] = q0 + t < a.seqlen ? __ldg(a.pos + static_cast<size_t>(b) * a.seqlen + q0 + t) : 0;
+}
+
+// Stages the rotary-table rows of tokens q0 .. q0+N-1 whose positions are p
+// (256 bytes each, consecutive in shared memory at `dst`), completing on
+// `bar`; tokens past the sequence end are skipped. Consecutive positions (the
+// usual p = token index) take one bulk copy, others one copy per row. Returns
+// the bytes requested. Run by one thread.
+template <int N>
+__device__ __forceinline__ uint32_t stage_rope_rows_at(const PrefillArgs& a, const int (&p)[N],
+                                                       int q0, uint32_t dst, uint32_t bar) {
+  constexpr uint32_t kRowBytes = kRopePairs * sizeof(float2);
+  const int n = min(N, a.seqlen - q0);
+  bool run = p[0] >= 0 && p[0] + n <= kMaxPosition;
+#pragma unroll
+  for (int t = 1; t < N; ++t) run = run && (t >= n || p[t] == p[0] + t);
+  if (run) {
+    bulk_load(dst, a.rope + static_cast<size_t>(p[0]) * kRopePairs, kRowBytes * n, bar);
+    return kRowBytes * n;
+  }
+#pragma unroll
+  for (int t = 0; t < N; ++t) {
+    if (t >= n) break;
+    int pt = p[t];
+    if (pt < 0 || pt >= kMaxPosition) {
+      atomicOr(a.err, kErrPosition);
+      pt = pt < 0 ? 0 : kMaxPosition - 1;
+    }
+    bulk_load(dst + t * kRowBytes, a.rope + static_cast<size_t>(pt) * kRopePairs, kRowBytes, bar);
+  }
+  return kRowBytes * n;
+}
+
 // S_m = Q_m K^T for one K/V tile (4 MMAs of K = 16 over head_dim 64).
 __device__ __forceinline__ void issue_qk(const Ctx& ctx, uint32_t tmem, int m, int qs, int s) {
   constexpr uint32_t idesc = idesc_bf16(128, kBlockN, false);
@@ -663,13 +702,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // (key index q_start+i) sees keys (i-W, i], so the whole item needs only the
 // 144 keys [q0-128, q0+16): one K/V span per item (TMA zero-fills rows before
 // 0 and past the last key), S = Q K^T with N = 144 and a single-tile softmax
-// (no online rescaling). Keys arrive already rotated; the RoPE warps rotate
-// the item's Q rows. Consecutive items alternate between the two softmax
-// warpgroups so the tensor core works on one item while the other's softmax
-// runs; the single issuer issues an item's Q K^T and the previous item's P V
-// in whichever order their inputs land. Each item's Q, K, V and table rows
-// share one ring stage; outputs go through a 3-slot staging ring so the store
-// of an item overlaps the next items' epilogues.
+// (no online rescaling). Keys arrive already rotated. Consecutive items
+// alternate between the two softmax warpgroups, and the warpgroup that owns an
+// item also rotates its Q rows (one row per thread) before waiting for S, so
+// the tensor core works on one item while the other's softmax runs; the single
+// issuer issues an item's Q K^T and the previous item's P V in whichever order
+// their inputs land. Each item's Q, K, V and table rows share one ring stage
+// (the producer loads each item's positions one item ahead and copies the
+// table rows of consecutive positions in one piece); outputs go through a
+// 3-slot staging ring so the store of an item overlaps the next items'
+// epilogues.
 namespace band {
 
 constexpr int kTokens = 16;
@@ -768,7 +810,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < band::kStages; ++s) {
       mbar_init(ctx.bar(band::BAR_QK_FULL + s), 1);
       mbar_init(ctx.bar(band::BAR_V_FULL + s), 1);
-      mbar_init(ctx.bar(band::BAR_READY + s), 2);
+      mbar_init(ctx.bar(band::BAR_READY + s), 4);
       mbar_init(ctx.bar(band::BAR_EMPTY + s), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -804,25 +846,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&maps.v_band);
         int k = 0;
         band::Item it;
-        for (; band::item_for(args, k, cta, &it); ++k) {
+        // Positions of an item's tokens are loaded one item ahead into the
+        // other of two register sets, so their round trip to memory hides
+        // behind the stage wait and the previous item's copies.
+        int pa[band::kTokens], pb[band::kTokens];
+        auto issue = [&](const band::Item& cur, const int (&p)[band::kTokens]) -> bool {
           const int s = k % band::kStages;
           if (k >= band::kStages &&
               !ctx.wait(band::BAR_EMPTY + s, ((k / band::kStages) - 1) & 1))
-            break;
-          const int kb = args.q_start + it.q0 - 128;  // span start, as a key index
+            return false;
+          const int kb = args.q_start + cur.q0 - 128;  // span start, as a key index
           const uint32_t tab_bytes =
-              kRopePairs * 8 * static_cast<uint32_t>(min(band::kTokens, S - it.q0));
+              kRopePairs * 8 * static_cast<uint32_t>(min(band::kTokens, S - cur.q0));
           mbar_arrive_expect_tx(ctx.bar(band::BAR_QK_FULL + s),
                                 band::kQBytes + band::kKVBytes + tab_bytes);
-          tma_load_4d(ctx.q(s), &maps.q, ctx.bar(band::BAR_QK_FULL + s), 0, it.g * kGroup, it.q0,
-                      it.b);
-          stage_rope_rows<band::kTokens, kRopePairs * 8>(args, it.b, it.q0, ctx.tab(s),
-                                                         ctx.bar(band::BAR_QK_FULL + s));
+          tma_load_4d(ctx.q(s), &maps.q, ctx.bar(band::BAR_QK_FULL + s), 0, cur.g * kGroup,
+                      cur.q0, cur.b);
+          stage_rope_rows_at<band::kTokens>(args, p, cur.q0, ctx.tab(s),
+                                            ctx.bar(band::BAR_QK_FULL + s));
           // rotated keys: see the same wait in prefill_kernel
           if (k == 0) griddep_wait();
-          tma_load_4d(ctx.k(s), &maps.k_band, ctx.bar(band::BAR_QK_FULL + s), 0, it.g, kb, it.b);
+          tma_load_4d(ctx.k(s), &maps.k_band, ctx.bar(band::BAR_QK_FULL + s), 0, cur.g, kb,
+                      cur.b);
           mbar_arrive_expect_tx(ctx.bar(band::BAR_V_FULL + s), band::kKVBytes);
-          tma_load_4d(ctx.v(s), &maps.v_band, ctx.bar(band::BAR_V_FULL + s), 0, it.g, kb, it.b);
+          tma_load_4d(ctx.v(s), &maps.v_band, ctx.bar(band::BAR_V_FULL + s), 0, cur.g, kb, cur.b);
+          ++k;
+          return true;
+        };
+        band::Item nx;
+        if (band::item_for(args, 0, cta, &it)) load_positions(args, it.b, it.q0, pa);
+        while (band::item_for(args, k, cta, &it)) {
+          if (band::item_for(args, k + 1, cta, &nx)) load_positions(args, nx.b, nx.q0, pb);
+          if (!issue(it, pa) || !band::item_for(args, k, cta, &it)) break;
+          if (band::item_for(args, k + 1, cta, &nx)) load_positions(args, nx.b, nx.q0, pa);
+          if (!issue(it, pb)) break;
         }
         if (*ctx.abort_flag) {
           volatile int never = 0;
@@ -903,27 +960,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         volatile int never = 0;
         mbar_wait(ctx.bar(band::BAR_MMA_DONE), 0, &never, nullptr, 0, kWaitTimeoutNs);
       }
-    } else {
-      // -------------------------------------------------------------- RoPE
-      const int t = static_cast<int>(threadIdx.x) - 64;  // 0..63
-      band::Item it;
-      bool ok = !skip;
-      for (int k = 0; ok && band::item_for(args, k, cta, &it); ++k) {
-        const int s = k % band::kStages;
-        if (!(ok = ctx.wait_warp(band::BAR_QK_FULL + s, (k / band::kStages) & 1))) break;
-        uint8_t* qt = smem + band::kOffStage + s * band::kStageBytes;
-        const float2* tab =
-            reinterpret_cast<const float2*>(qt + band::kQBytes + 2 * band::kKVBytes);
-#pragma unroll 1
-        for (int rr = 0; rr < 2; ++rr) {
-          const int row = t + 64 * rr;
-          if (it.q0 + (row >> 3) < S) rope_row(qt + row * 128, row, tab + (row >> 3) * kRopePairs);
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(ctx.bar(band::BAR_READY + s));
-      }
     }
+    // warps 2-3 have no role here (the softmax warpgroups rotate Q)
   } else if (wg == 1 || wg == 2) {
     // ---------------------------------------------------------------- softmax
     setmaxnreg_inc<band::kRegsSoftmax>();
@@ -944,6 +982,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int c_hi = d + 128;
       const float sink = __ldg(args.sinks + it.g * kGroup + (r & 7));
       const bool sink_off = isinf(sink) && sink < 0.f;
+      {
+        // RoPE of this item's Q: row r (token d, head r % 8) of the stage's Q tile
+        const int s = k % band::kStages;
+        if (!(ok = ctx.wait_warp(band::BAR_QK_FULL + s, (k / band::kStages) & 1))) break;
+        uint8_t* qt = smem + band::kOffStage + s * band::kStageBytes;
+        if (it.q0 + d < S)
+          rope_row(qt + r * 128, r,
+                   reinterpret_cast<const float2*>(qt + band::kQBytes + 2 * band::kKVBytes) +
+                       d * kRopePairs);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ctx.bar(band::BAR_READY + s));
+      }
       if (!(ok = ctx.wait_warp(band::BAR_S_FULL + m, i & 1))) break;
       tc_fence_after_sync();
       uint32_t sv[band::kSpan];
