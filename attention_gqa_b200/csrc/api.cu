@@ -462,7 +462,11 @@ int gptoss_attn_prefill_backward(const void* q, const void* k, const void* v, co
   a.window = (window > 0 && window < seqlen) ? window : 0;
   a.n_qt = backward_q_tiles(seqlen);
   const int sms = g_state[dev].num_sms;
+  // the per-row arrays' padding tile is read (and masked) by the last dK/dV steps
+  const size_t rows = static_cast<size_t>(batch) * seqlen * kNumHeads;
   if (cudaMemsetAsync(dsinks, 0, kNumHeads * sizeof(float), stream) != cudaSuccess ||
+      cudaMemsetAsync(a.lse2 + rows, 0, 128 * sizeof(float), stream) != cudaSuccess ||
+      cudaMemsetAsync(a.dd + rows, 0, 128 * sizeof(float), stream) != cudaSuccess ||
       launch_rope_rows(q, pos, a.rope, ws + off[0], batch, seqlen, seqlen, 0, kNumHeads, sms * 8,
                        a.err, stream) != cudaSuccess ||
       launch_rope_rows(k, pos, a.rope, ws + off[1], batch, seqlen, seqlen, 0, kNumKvHeads,

@@ -484,7 +484,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
             const int tt = col >> 3;
             const bool vis = tt >= lo_t && tt <= hi_t;
             p[u] = vis ? ex2_approx(__uint_as_float(sv[e + u]) * kScaleLog2 - ld[col]) : 0.f;
-            ds[u] = p[u] * (__uint_as_float(pv[e + u]) - ld[64 + col]) * kScale;
+            // rows past the sequence carry no lse or D: keep them out of dK
+            ds[u] = vis ? p[u] * (__uint_as_float(pv[e + u]) - ld[64 + col]) * kScale : 0.f;
           }
           pw[e / 2] = pack_bf16x2(p[0], p[1]);
           dw[e / 2] = pack_bf16x2(ds[0], ds[1]);

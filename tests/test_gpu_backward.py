@@ -108,3 +108,25 @@ def test_lse_matches_the_forward(cuda_device):
         f = synth.bf16_bits_to_f64
         lref = _lse_ref(f(x["q"]), f(x["k"]), x["sinks"], x["pos"], window)
         assert np.max(np.abs(lse.double().cpu().numpy() - lref)) < 3e-2, window
+
+
+def test_backward_ignores_workspace_contents(cuda_device):
+    """The workspace needs no initialisation: a NaN-filled one gives the same
+    gradients (the per-row arrays' padding, read by the last dK/dV steps of a
+    sequence whose length is not a multiple of 8, is cleared by the call)."""
+    B, S, window = 1, 77, 0
+    x = synth.make_prefill_inputs(230, 0, B, S)
+    q, k, v = bits_to_dev(x["q"]), bits_to_dev(x["k"]), bits_to_dev(x["v"])
+    sinks, pos = torch.from_numpy(x["sinks"]).cuda(), torch.from_numpy(x["pos"]).cuda()
+    out, lse = gqa.prefill_lse(q, k, v, sinks, pos, window)
+    dout = bits_to_dev(synth.bf16_normal(0xD7, (B, S, NQ, D)))
+    clean = gqa.prefill_backward(q, k, v, sinks, pos, window, out, lse, dout)
+    nbytes = gqa.prefill_backward_workspace_bytes(B, S)
+    ws = torch.full((nbytes // 4,), float("nan"), dtype=torch.float32, device="cuda")
+    dirty = gqa.prefill_backward(q, k, v, sinks, pos, window, out, lse, dout,
+                                 workspace=ws.view(torch.uint8))
+    gqa.check()
+    for a, b in zip(clean[:3], dirty[:3]):
+        assert torch.isfinite(b.float()).all()
+        assert torch.equal(a, b)
+    assert torch.isfinite(dirty[3]).all()
