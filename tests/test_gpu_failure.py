@@ -61,3 +61,39 @@ def test_kernels_skip_work_while_a_timeout_is_pending(cuda_device):
         ref = oracle.decode(synth.bf16_bits_to_f64(d["q"]), synth.bf16_bits_to_f64(d["kcache"]),
                             synth.bf16_bits_to_f64(d["vcache"]), d["sinks"], d["len"], window)
         compare(dev_to_f64(dout), ref, "decode after clear W=%d" % window)
+
+
+@pytest.mark.gpu
+def test_backward_skips_work_while_a_timeout_is_pending(cuda_device):
+    """The dQ and dK/dV kernels check the error word at start-up like the
+    forward kernels: launched while a timeout is pending they leave the
+    gradients untouched; after the clear the same call gives the gradients."""
+    lib = gqa._load()
+    stream = torch.cuda.current_stream().cuda_stream
+    x = synth.make_prefill_inputs(3, 1, 1, 80)
+    q, k, v = bits_to_dev(x["q"]), bits_to_dev(x["k"]), bits_to_dev(x["v"])
+    sinks, pos = torch.from_numpy(x["sinks"]).cuda(), torch.from_numpy(x["pos"]).cuda()
+    out, lse = gqa.prefill_lse(q, k, v, sinks, pos, 0)
+    dout = bits_to_dev(synth.bf16_normal(0xD9, (1, 80, 64, 64)))
+    ref = gqa.prefill_backward(q, k, v, sinks, pos, 0, out, lse, dout)
+    gqa.check()
+    ws = torch.empty(gqa.prefill_backward_workspace_bytes(1, 80), dtype=torch.uint8, device="cuda")
+
+    def nan_like(t):
+        return torch.full(t.shape, float("nan"), dtype=t.dtype, device="cuda")
+    grads = [nan_like(t) for t in ref[:3]] + [torch.zeros(64, device="cuda")]
+
+    def call():
+        return lib.gptoss_attn_prefill_backward(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), sinks.data_ptr(), pos.data_ptr(), 0,
+            out.data_ptr(), lse.data_ptr(), dout.data_ptr(), grads[0].data_ptr(),
+            grads[1].data_ptr(), grads[2].data_ptr(), grads[3].data_ptr(), 1, 80, ws.data_ptr(),
+            ws.numel(), stream)
+    assert lib.gptoss_attn_debug_wait_timeout(1000, stream) == 0
+    assert call() == 0
+    assert lib.gptoss_attn_check(stream) == DEVICE_TIMEOUT
+    assert all(torch.isnan(g.float()).all() for g in grads[:3])
+    assert call() == 0
+    gqa.check()
+    for g, r in zip(grads[:3], ref[:3]):
+        assert torch.equal(g, r)
