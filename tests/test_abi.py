@@ -188,3 +188,67 @@ def test_decode_noalloc_binding_checks_shapes_before_the_library(monkeypatch):
     # well-formed host tensors pass the shape checks and are refused as not on a device
     with pytest.raises(ValueError, match="device tensors"):
         gqa.decode_noalloc(*good.values(), 0)
+
+
+def test_yarn_entry_points_argument_errors(lib):
+    """The _yarn entry points validate exactly like the plain ones, and the YaRN
+    decode refuses caches longer than the table's 131072 positions. Every call
+    here has one bad argument, so none reaches a device."""
+    c = _header_codes()
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    fp = lib.gptoss_attn_prefill_yarn
+    fp.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, vp, sz, vp]
+    need = lib.gptoss_attn_prefill_workspace_bytes(1, 8)
+    assert fp(None, 32, 48, 64, 80, 0, 96, 1, 8, 112, need, None) == c["GPTOSS_ATTN_ERR_NULL_PTR"]
+    assert fp(16, 32, 48, 64, 80, 0, 96, 1, 131073, 112, need, None) == \
+        c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert fp(16, 40, 48, 64, 80, 0, 96, 1, 8, 112, need, None) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
+    assert fp(16, 32, 48, 64, 80, 0, 96, 1, 8, 112, need - 1, None) == \
+        c["GPTOSS_ATTN_ERR_SMALL_WORKSPACE"]
+    fd = lib.gptoss_attn_decode_yarn
+    fd.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, vp, sz, vp]
+    big = 131073
+    wsb = lib.gptoss_attn_decode_workspace_bytes(1, big, 0)
+    assert fd(16, 32, 48, 64, 80, 0, 96, 1, big, 128, wsb, None) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert fd(16, 32, None, 64, 80, 0, 96, 1, 64, 128, 1 << 20, None) == \
+        c["GPTOSS_ATTN_ERR_NULL_PTR"]
+
+
+def test_training_entry_points_argument_errors(lib):
+    """gptoss_attn_prefill_lse and gptoss_attn_prefill_backward reject bad
+    arguments on the host, and the backward workspace is sized as declared."""
+    c = _header_codes()
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    fl = lib.gptoss_attn_prefill_lse
+    fl.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, vp, sz, vp]
+    need = lib.gptoss_attn_prefill_workspace_bytes(1, 8)
+    assert fl(16, 32, 48, 64, 80, 0, 96, None, 1, 8, 112, need, None) == \
+        c["GPTOSS_ATTN_ERR_NULL_PTR"]
+    assert fl(16, 32, 48, 64, 80, 0, 96, 130, 1, 8, 112, need, None) == \
+        c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
+    wb = lib.gptoss_attn_prefill_backward_workspace_bytes
+    wb.argtypes = [i32, i32]
+    wb.restype = sz
+    assert wb(0, 8) == 0 and wb(1, 0) == 0 and wb(1, 131073) == 0
+
+    def r256(x):
+        return (x + 255) // 256 * 256
+    B, S = 2, 100
+    rows = B * S * 64
+    assert wb(B, S) == r256(rows * 64 * 2) + r256(B * S * 8 * 64 * 2) + 2 * r256((rows + 128) * 4)
+    fb = lib.gptoss_attn_prefill_backward
+    fb.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, sz, vp]
+    ok = dict(q=16, k=32, v=48, s=64, p=80, w=0, o=96, lse=112, do=128, dq=144, dk=160,
+              dv=176, ds=192, b=B, S=S, ws=208, n=wb(B, S))
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return fb(a["q"], a["k"], a["v"], a["s"], a["p"], a["w"], a["o"], a["lse"], a["do"],
+                  a["dq"], a["dk"], a["dv"], a["ds"], a["b"], a["S"], a["ws"], a["n"], None)
+    for name in ("q", "lse", "do", "dq", "dk", "dv", "ds", "ws"):
+        assert call(**{name: None}) == c["GPTOSS_ATTN_ERR_NULL_PTR"], name
+    assert call(b=0) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert call(S=0) == c["GPTOSS_ATTN_ERR_BAD_SHAPE"]
+    assert call(dk=168) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
+    assert call(ds=194) == c["GPTOSS_ATTN_ERR_BAD_ALIGN"]
+    assert call(n=wb(B, S) - 1) == c["GPTOSS_ATTN_ERR_SMALL_WORKSPACE"]
