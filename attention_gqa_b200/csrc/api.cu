@@ -162,7 +162,7 @@ static int prefill_impl(const void* q, const void* k, const void* v, const float
   const uint64_t kstr[3] = {kHeadDim * 2, kNumKvHeads * kHeadDim * 2,
                             S * kNumKvHeads * kHeadDim * 2};
   const uint32_t kbox[4] = {kHeadDim, 1, 128, 1};
-  const uint32_t kbox_band[4] = {kHeadDim, 1, 144, 1};
+  const uint32_t kbox_band[4] = {kHeadDim, 1, 16, 1};  // 16-key blocks of the band kernel
   // the attention kernels read the rotated keys from the workspace
   if (!make_tmap_bf16_4d(&maps.q, q, qdims, qstr, qbox) ||
       !make_tmap_bf16_4d(&maps.o, out, qdims, qstr, qbox) ||
@@ -226,7 +226,7 @@ static int prefill_chunk_impl(const void* q, const void* k, const void* v, const
   const uint64_t cstr[3] = {kHeadDim * 2, kNumKvHeads * kHeadDim * 2,
                             L * kNumKvHeads * kHeadDim * 2};
   const uint32_t kbox[4] = {kHeadDim, 1, 128, 1};
-  const uint32_t kbox_band[4] = {kHeadDim, 1, 144, 1};
+  const uint32_t kbox_band[4] = {kHeadDim, 1, 16, 1};  // 16-key blocks of the band kernel
   if (!make_tmap_bf16_4d(&maps.q, q, qdims, qstr, qbox) ||
       !make_tmap_bf16_4d(&maps.o, out, qdims, qstr, qbox) ||
       !make_tmap_bf16_4d(&maps.k, kcache, cdims, cstr, kbox) ||

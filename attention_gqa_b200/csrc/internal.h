@@ -47,7 +47,7 @@ struct PrefillArgs {
 
 struct PrefillMaps {
   CUtensorMap q, k, v, o;   // q/o boxes (64, 8, 16, 1); k/v boxes (64, 1, 128, 1)
-  CUtensorMap k_band, v_band;  // k/v boxes (64, 1, 144, 1) for the narrow-band kernel
+  CUtensorMap k_band, v_band;  // k/v boxes (64, 1, 16, 1): key blocks of the narrow-band kernel
 };
 
 // True when the narrow-band kernel (0 < window <= 128) serves the layer.
