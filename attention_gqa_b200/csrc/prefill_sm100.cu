@@ -732,7 +732,7 @@ namespace band {
 constexpr int kTokens = 16;
 constexpr int kSpan = 144;  // 128 keys before the tile + the tile's 16
 constexpr int kSpanBlocks = kSpan / 16;
-constexpr int kQSlots = 6;
+constexpr int kQSlots = 4;
 constexpr int kRing = 18;  // key/value blocks of 16 keys
 // Register budgets after the warpgroup split (launch is 512 x 128): the
 // softmax rows here are 144 scores wide, so it gets more than in prefill_kernel.
