@@ -52,6 +52,8 @@ struct PrefillMaps {
 
 // True when the narrow-band kernel (0 < window <= 128) serves the layer.
 bool prefill_uses_band(int window);
+// Query tokens per work item of the narrow-band kernel.
+constexpr int kBandTokens = 16;
 // Work items of one prefill launch.
 int prefill_items(int batch, int seqlen, int window);
 // Item order of the full-causal kernel for these sizes (PrefillArgs::order_chunk).
@@ -59,6 +61,9 @@ int prefill_order_chunk(int batch, int keys, int grid);
 
 // Launches the prefill kernel; returns a cudaError_t.
 cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillArgs& args, cudaStream_t stream);
+// Launches the narrow-band kernel on `grid` CTAs (called by launch_prefill).
+cudaError_t launch_prefill_band(const PrefillMaps& maps, const PrefillArgs& args, int grid,
+                                cudaStream_t stream);
 
 // Diagnostic: a bounded wait on a barrier nothing arrives at (sets kErrTimeout).
 cudaError_t launch_wait_timeout(int* err, uint64_t timeout_ns, cudaStream_t stream);

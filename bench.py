@@ -97,9 +97,13 @@ def load_peaks():
 
 
 def source_digest() -> str:
-    p = os.path.join(ROOT, "attention_gqa_b200", "csrc", "prefill_sm100.cu")
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Digest of the full-causal prefill kernel's sources (kernel file and the
+    header it shares with the narrow-band kernel)."""
+    h = hashlib.sha256()
+    for name in ("prefill_sm100.cu", "prefill_common.cuh"):
+        with open(os.path.join(ROOT, "attention_gqa_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def profiled_traffic(path: str):
