@@ -378,23 +378,26 @@ int gptoss_attn_decode_yarn(const void* q, const void* kcache, const void* vcach
                      workspace_bytes, stream, Rope::kYarn);
 }
 
-// Backward workspace: rotated q, rotated k, then lse2 and D in [b][g][t][8]
-// layout, each float array padded by one 128-row tile.
+// Backward workspace: rotated q, rotated k, lse2 and D in [b][g][t][8] layout
+// (each float array padded by one 128-row tile), then the fp32 sums of dK'
+// and dV ([b][t][g][64] each).
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-static void backward_layout(int batch, int seqlen, size_t off[5]) {
+static void backward_layout(int batch, int seqlen, size_t off[7]) {
   const size_t BS = static_cast<size_t>(batch) * seqlen;
   off[0] = 0;
   off[1] = align256(BS * kNumHeads * kHeadDim * 2);
   off[2] = off[1] + align256(BS * kNumKvHeads * kHeadDim * 2);
   off[3] = off[2] + align256((BS * kNumHeads + 128) * 4);
   off[4] = off[3] + align256((BS * kNumHeads + 128) * 4);
+  off[5] = off[4] + align256(BS * kNumKvHeads * kHeadDim * 4);
+  off[6] = off[5] + align256(BS * kNumKvHeads * kHeadDim * 4);
 }
 
 size_t gptoss_attn_prefill_backward_workspace_bytes(int batch, int seqlen) {
   if (batch < 1 || seqlen < 1 || seqlen > kMaxPosition || batch > 65535) return 0;
-  size_t off[5];
+  size_t off[7];
   backward_layout(batch, seqlen, off);
-  return off[4];
+  return off[6];
 }
 
 int gptoss_attn_prefill_backward(const void* q, const void* k, const void* v, const float* sinks,
@@ -419,7 +422,7 @@ int gptoss_attn_prefill_backward(const void* q, const void* k, const void* v, co
   if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, Rope::kPlain);
   if (st != GPTOSS_ATTN_OK) return st;
 
-  size_t off[5];
+  size_t off[7];
   backward_layout(batch, seqlen, off);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   BackwardMaps maps;
@@ -457,14 +460,20 @@ int gptoss_attn_prefill_backward(const void* q, const void* k, const void* v, co
   a.dq = static_cast<uint16_t*>(dq);
   a.dk = static_cast<uint16_t*>(dk);
   a.dv = static_cast<uint16_t*>(dv);
+  a.dk32 = reinterpret_cast<float*>(ws + off[4]);
+  a.dv32 = reinterpret_cast<float*>(ws + off[5]);
   a.batch = batch;
   a.seqlen = seqlen;
   a.window = (window > 0 && window < seqlen) ? window : 0;
   a.n_qt = backward_q_tiles(seqlen);
   const int sms = g_state[dev].num_sms;
+  // dK/dV work in about four waves of two CTAs per SM
+  backward_plan(&a, 8 * sms);
   // the per-row arrays' padding tile is read (and masked) by the last dK/dV steps
   const size_t rows = static_cast<size_t>(batch) * seqlen * kNumHeads;
   if (cudaMemsetAsync(dsinks, 0, kNumHeads * sizeof(float), stream) != cudaSuccess ||
+      (a.kv_chunks > 1 &&
+       cudaMemsetAsync(ws + off[4], 0, off[6] - off[4], stream) != cudaSuccess) ||
       cudaMemsetAsync(a.lse2 + rows, 0, 128 * sizeof(float), stream) != cudaSuccess ||
       cudaMemsetAsync(a.dd + rows, 0, 128 * sizeof(float), stream) != cudaSuccess ||
       launch_rope_rows(q, pos, a.rope, ws + off[0], batch, seqlen, seqlen, 0, kNumHeads, sms * 8,

@@ -24,17 +24,25 @@
 //     fp32 in TMEM), dS by the elementwise warpgroup (bf16 back into S's
 //     columns), dQ += dS K' (A from TMEM). dQ stays in TMEM until the item's
 //     end, is rotated back and stored as bf16.
-//   bwd_dkv_kernel: one CTA per (b, g, 128 keys) = M=128 keys; over the
-//     8-token (64-row) query tiles that see them: S^T = K'Q'^T, dP^T = V dO^T,
-//     P^T and dS^T by the elementwise warpgroup, dV += P^T dO and dK += dS^T Q'
-//     (A from TMEM, summing over the 8 heads of the group because they are
-//     rows of the tile). No atomics on dq, dk or dv.
+//   bwd_dkv_kernel: one CTA per (b, g, 128 keys, chunk of query steps) = M=128
+//     keys; over its 8-token (64-row) query steps that see them: S^T = K'Q'^T,
+//     dP^T = V dO^T, P^T and dS^T by the elementwise warpgroup, dV += P^T dO and
+//     dK += dS^T Q' (A from TMEM, summing over the 8 heads of the group because
+//     they are rows of the tile). A key tile's steps are split into chunks of
+//     similar length, so the first key tiles of a causal sequence (which see
+//     every query) do not set the kernel's length; each chunk adds its fp32
+//     dK', dV to zeroed sums in the workspace (vector reductions). When every
+//     tile fits one chunk (long sequences, sliding windows) the CTA writes
+//     dk = R(pos)^T dK' and dv as bf16 itself.
+//   bwd_dkv_finish_kernel (split tiles only): dk = R(pos)^T dK' and dv from the
+//     sums, as bf16.
 // Each CTA takes 256 tensor-memory columns and ~100 KB of shared memory, so
 // two CTAs share an SM and one's elementwise work overlaps the other's MMAs.
 // Roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
 // warps 2-5 the elementwise warpgroup (thread = TMEM lane; warp w reads lanes
 // 32 (w % 4) .. 32 (w % 4) + 31).
 // Every pipeline wait is bounded like the forward kernels'.
+#include <algorithm>
 #include <cmath>
 
 #include "internal.h"
@@ -176,6 +184,26 @@ __device__ __forceinline__ void unrotate_store(const uint32_t (&lo)[32], const u
   for (int i = 0; i < 8; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
 }
 
+// Adds 4 floats to global memory at p (16-byte aligned) with one vector reduction.
+__device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+// Adds a thread's 64-float accumulator row (lo: columns 0-31, hi: 32-63) to `row`.
+__device__ __forceinline__ void red_add_row(float* row, const uint32_t (&lo)[32],
+                                            const uint32_t (&hi)[32]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    red_add4(row + 4 * i, __uint_as_float(lo[4 * i]), __uint_as_float(lo[4 * i + 1]),
+             __uint_as_float(lo[4 * i + 2]), __uint_as_float(lo[4 * i + 3]));
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    red_add4(row + 32 + 4 * i, __uint_as_float(hi[4 * i]), __uint_as_float(hi[4 * i + 1]),
+             __uint_as_float(hi[4 * i + 2]), __uint_as_float(hi[4 * i + 3]));
+}
+
 __device__ __forceinline__ int clamp_pos(int p, int* err) {
   if (p < 0 || p >= kMaxPosition) {
     atomicOr(err, kErrPosition);
@@ -231,6 +259,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  // the dK/dV kernel does not read this kernel's results: let it start filling
+  // the SMs this grid's last CTAs leave idle
+  griddep_launch_dependents();
   Ctx ctx;
   const uint32_t tmem = setup(ctx, smem, kQOffBar, a.err);
   const bool skip = *ctx.abort_flag != 0;
@@ -364,10 +395,25 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
   teardown(tmem);
 }
 
-// dK and dV for one (b, g, 128-key) tile per CTA.
+// Partial dK and dV for one (b, g, 128-key tile, chunk of query steps) per CTA.
 __global__ void __launch_bounds__(bwd::kThreads, 2)
     bwd_dkv_kernel(const __grid_constant__ BackwardMaps maps, const BackwardArgs a) {
   using namespace bwd;
+  const int S = a.seqlen, W = a.window;
+  // chunk-major, then key tile, then (b, g): full chunks of all tiles first
+  const int per_tile = kNumKvHeads * a.batch;
+  const int n_kt = (S + kKeys - 1) / kKeys;
+  const int idx = static_cast<int>(blockIdx.x);
+  const int chunk = idx / (n_kt * per_tile);
+  const int kt = (idx / per_tile) % n_kt;
+  const int g = (idx % per_tile) % kNumKvHeads, b = (idx % per_tile) / kNumKvHeads;
+  const int kb = kt * kKeys;
+  // query tokens that see a key of this tile: [kb, t_max], in 8-token steps
+  const int t_max = W > 0 ? min(S - 1, kb + kKeys - 1 + W - 1) : S - 1;
+  const int j0 = chunk * a.kv_steps;
+  const int qt0 = kb / kKTok + j0;  // this CTA's first step
+  const int n_tiles = min(t_max / kKTok - kb / kKTok + 1 - j0, a.kv_steps);
+  if (n_tiles <= 0) return;  // the tile has fewer chunks than the longest one
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -375,17 +421,6 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
   const uint32_t tmem = setup(ctx, smem, kKOffBar, a.err);
   const bool skip = *ctx.abort_flag != 0;
   const int warp = static_cast<int>(threadIdx.x >> 5), lane = static_cast<int>(threadIdx.x & 31);
-  const int S = a.seqlen, W = a.window;
-  // longest first: key tiles from the start of the sequence
-  const int per_tile = kNumKvHeads * a.batch;
-  const int idx = static_cast<int>(blockIdx.x);
-  const int kt = idx / per_tile;
-  const int g = (idx % per_tile) % kNumKvHeads, b = (idx % per_tile) / kNumKvHeads;
-  const int kb = kt * kKeys;
-  // query tokens that see a key of this tile: [kb, t_max]
-  const int t_max = W > 0 ? min(S - 1, kb + kKeys - 1 + W - 1) : S - 1;
-  const int qt0 = kb / kKTok;
-  const int n_tiles = t_max / kKTok - qt0 + 1;
   const float* lse2_g = a.lse2 + (static_cast<int64_t>(b) * kNumKvHeads + g) * S * kGroup;
   const float* dd_g = a.dd + (static_cast<int64_t>(b) * kNumKvHeads + g) * S * kGroup;
 
@@ -501,39 +536,107 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
     if (ok && (ok = ctx.wait_warp(BAR_ACC_FULL, 0))) {
       tc_fence_after_sync();
       uint32_t lo[32], hi[32];
+      const int64_t row = ((static_cast<int64_t>(b) * S + kj) * kNumKvHeads + g) * kHeadDim;
       tmem_ld32(tmem + lane_off + kColA, lo);
       tmem_ld32(tmem + lane_off + kColA + 32, hi);
       if (kj < S) {
-        uint4* dv4 = reinterpret_cast<uint4*>(
-            a.dv + ((static_cast<int64_t>(b) * S + kj) * kNumKvHeads + g) * kHeadDim);
+        if (a.kv_chunks > 1) {
+          red_add_row(a.dv32 + row, lo, hi);
+        } else {
+          // the only chunk of the tile: dv straight to bf16
+          uint4* dv4 = reinterpret_cast<uint4*>(a.dv + row);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          dv4[i] = make_uint4(pack_bf16x2(__uint_as_float(lo[8 * i]), __uint_as_float(lo[8 * i + 1])),
-                              pack_bf16x2(__uint_as_float(lo[8 * i + 2]), __uint_as_float(lo[8 * i + 3])),
-                              pack_bf16x2(__uint_as_float(lo[8 * i + 4]), __uint_as_float(lo[8 * i + 5])),
-                              pack_bf16x2(__uint_as_float(lo[8 * i + 6]), __uint_as_float(lo[8 * i + 7])));
-          dv4[4 + i] = make_uint4(pack_bf16x2(__uint_as_float(hi[8 * i]), __uint_as_float(hi[8 * i + 1])),
-                                  pack_bf16x2(__uint_as_float(hi[8 * i + 2]), __uint_as_float(hi[8 * i + 3])),
-                                  pack_bf16x2(__uint_as_float(hi[8 * i + 4]), __uint_as_float(hi[8 * i + 5])),
-                                  pack_bf16x2(__uint_as_float(hi[8 * i + 6]), __uint_as_float(hi[8 * i + 7])));
+          for (int i = 0; i < 4; ++i) {
+            dv4[i] = make_uint4(
+                pack_bf16x2(__uint_as_float(lo[8 * i]), __uint_as_float(lo[8 * i + 1])),
+                pack_bf16x2(__uint_as_float(lo[8 * i + 2]), __uint_as_float(lo[8 * i + 3])),
+                pack_bf16x2(__uint_as_float(lo[8 * i + 4]), __uint_as_float(lo[8 * i + 5])),
+                pack_bf16x2(__uint_as_float(lo[8 * i + 6]), __uint_as_float(lo[8 * i + 7])));
+            dv4[4 + i] = make_uint4(
+                pack_bf16x2(__uint_as_float(hi[8 * i]), __uint_as_float(hi[8 * i + 1])),
+                pack_bf16x2(__uint_as_float(hi[8 * i + 2]), __uint_as_float(hi[8 * i + 3])),
+                pack_bf16x2(__uint_as_float(hi[8 * i + 4]), __uint_as_float(hi[8 * i + 5])),
+                pack_bf16x2(__uint_as_float(hi[8 * i + 6]), __uint_as_float(hi[8 * i + 7])));
+          }
         }
       }
       tmem_ld32(tmem + lane_off + kColB, lo);
       tmem_ld32(tmem + lane_off + kColB + 32, hi);
       if (kj < S) {
-        const int p = bwd::clamp_pos(__ldg(a.pos + static_cast<int64_t>(b) * S + kj), a.err);
-        unrotate_store(lo, hi, a.rope + static_cast<size_t>(p) * kRopePairs,
-                       a.dk + ((static_cast<int64_t>(b) * S + kj) * kNumKvHeads + g) * kHeadDim);
+        if (a.kv_chunks > 1) {
+          red_add_row(a.dk32 + row, lo, hi);
+        } else {
+          const int p = bwd::clamp_pos(__ldg(a.pos + static_cast<int64_t>(b) * S + kj), a.err);
+          unrotate_store(lo, hi, a.rope + static_cast<size_t>(p) * kRopePairs, a.dk + row);
+        }
       }
     }
   }
   teardown(tmem);
 }
 
+// dk = R(pos)^T dK' and dv from the fp32 sums, as bf16: one thread per
+// (token, kv head) row, grid-stride. Skipped while the error word holds a
+// timeout (the dK/dV CTAs then left the sums incomplete).
+__global__ void __launch_bounds__(256) bwd_dkv_finish_kernel(const BackwardArgs a) {
+  // like the other kernels, skip the work while a timeout is pending
+  if (*reinterpret_cast<volatile int*>(a.err) & kErrTimeout) return;
+  const int64_t n = static_cast<int64_t>(a.batch) * a.seqlen * kNumKvHeads;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; r < n;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4* k4 = reinterpret_cast<const float4*>(a.dk32 + r * kHeadDim);
+    const float4* v4 = reinterpret_cast<const float4*>(a.dv32 + r * kHeadDim);
+    uint32_t lo[32], hi[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 x = k4[i], y = k4[8 + i];
+      lo[4 * i] = __float_as_uint(x.x);
+      lo[4 * i + 1] = __float_as_uint(x.y);
+      lo[4 * i + 2] = __float_as_uint(x.z);
+      lo[4 * i + 3] = __float_as_uint(x.w);
+      hi[4 * i] = __float_as_uint(y.x);
+      hi[4 * i + 1] = __float_as_uint(y.y);
+      hi[4 * i + 2] = __float_as_uint(y.z);
+      hi[4 * i + 3] = __float_as_uint(y.w);
+    }
+    const int64_t bt = r / kNumKvHeads;  // b * S + t
+    const int p = bwd::clamp_pos(__ldg(a.pos + bt), a.err);
+    bwd::unrotate_store(lo, hi, a.rope + static_cast<size_t>(p) * kRopePairs, a.dk + r * kHeadDim);
+    uint4* d4 = reinterpret_cast<uint4*>(a.dv + r * kHeadDim);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 x = v4[2 * i], y = v4[2 * i + 1];
+      d4[i] = make_uint4(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w), pack_bf16x2(y.x, y.y),
+                         pack_bf16x2(y.z, y.w));
+    }
+  }
+}
+
 }  // namespace
 
 int backward_q_tiles(int seqlen) { return (seqlen + bwd::kTok - 1) / bwd::kTok; }
 int backward_k_tiles(int seqlen) { return (seqlen + bwd::kKeys - 1) / bwd::kKeys; }
+
+void backward_plan(BackwardArgs* a, int target_ctas) {
+  const int S = a->seqlen, W = a->window, n_kt = backward_k_tiles(S);
+  int64_t total = 0;
+  int longest = 1;
+  for (int kt = 0; kt < n_kt; ++kt) {
+    const int kb = kt * bwd::kKeys;
+    const int t_max = W > 0 ? std::min(S - 1, kb + bwd::kKeys - 1 + W - 1) : S - 1;
+    const int n = t_max / bwd::kKTok - kb / bwd::kKTok + 1;
+    total += n;
+    longest = std::max(longest, n);
+  }
+  total *= static_cast<int64_t>(kNumKvHeads) * a->batch;
+  // at least 32 steps per CTA (256 query tokens), so the partial sums stay a
+  // small share of the traffic
+  int64_t steps = (total + target_ctas - 1) / target_ctas;
+  if (steps < 32) steps = 32;
+  if (steps > longest) steps = longest;
+  a->kv_steps = static_cast<int>(steps);
+  a->kv_chunks = (longest + a->kv_steps - 1) / a->kv_steps;
+}
 
 cudaError_t launch_backward(const BackwardMaps& maps, const BackwardArgs& args, int num_sms,
                             cudaStream_t stream) {
@@ -553,9 +656,27 @@ cudaError_t launch_backward(const BackwardMaps& maps, const BackwardArgs& args, 
   bwd_dq_kernel<<<n_dq, bwd::kThreads, bwd::kSmemBytes, stream>>>(maps, args);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const unsigned n_dkv =
-      static_cast<unsigned>(backward_k_tiles(args.seqlen) * kNumKvHeads * args.batch);
-  bwd_dkv_kernel<<<n_dkv, bwd::kThreads, bwd::kSmemBytes, stream>>>(maps, args);
+  const unsigned n_dkv = static_cast<unsigned>(backward_k_tiles(args.seqlen) * kNumKvHeads *
+                                              args.batch * args.kv_chunks);
+  // programmatic dependent launch: independent of the dQ kernel, it overlaps
+  // that kernel's tail (both read only the preparation kernel's results, which
+  // are complete before the dQ kernel starts)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_dkv);
+  cfg.blockDim = dim3(bwd::kThreads);
+  cfg.dynamicSmemBytes = bwd::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, bwd_dkv_kernel, maps, args);
+  if (e != cudaSuccess || args.kv_chunks == 1) return e;
+  const int64_t rows = static_cast<int64_t>(args.batch) * args.seqlen * kNumKvHeads;
+  int64_t fin_blocks = (rows + 255) / 256;
+  if (fin_blocks > 8 * num_sms) fin_blocks = 8 * num_sms;
+  bwd_dkv_finish_kernel<<<static_cast<unsigned>(fin_blocks), 256, 0, stream>>>(args);
   return cudaGetLastError();
 }
 

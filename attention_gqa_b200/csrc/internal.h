@@ -118,10 +118,15 @@ struct BackwardArgs {
   uint16_t* dq;            // [B][S][64][64] bf16
   uint16_t* dk;            // [B][S][8][64] bf16
   uint16_t* dv;            // [B][S][8][64] bf16
+  float* dk32;             // workspace [B][S][8][64], zeroed: sums of dK' (rotated frame)
+  float* dv32;             // workspace [B][S][8][64], zeroed: sums of dV
   int batch;
   int seqlen;
   int window;              // <= 0: full causal
   int n_qt;                // 16-token query tiles per sequence
+  int kv_steps;            // 8-token query steps per dK/dV CTA (a key tile's steps are
+                           // split over several CTAs whose partial sums are added)
+  int kv_chunks;           // dK/dV CTAs per key tile (the most any tile needs)
 };
 
 struct BackwardMaps {
@@ -133,6 +138,9 @@ struct BackwardMaps {
 
 int backward_q_tiles(int seqlen);
 int backward_k_tiles(int seqlen);
+// Splits the dK/dV work: sets args->kv_steps and args->kv_chunks so that about
+// `target_ctas` CTAs of similar length cover every key tile's query steps.
+void backward_plan(BackwardArgs* args, int target_ctas);
 // Launches the preparation, dQ and dK/dV kernels (dsinks must be zeroed and
 // the rotated q and k written to the workspace before).
 cudaError_t launch_backward(const BackwardMaps& maps, const BackwardArgs& args, int num_sms,

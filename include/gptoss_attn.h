@@ -158,8 +158,9 @@ int gptoss_attn_prefill_lse(const void* q, const void* k, const void* v, const f
 
 /*
  * Bytes of device workspace gptoss_attn_prefill_backward() needs: the rotated
- * queries and keys (bf16) and two fp32 values per query row, plus alignment.
- * Returns 0 for invalid sizes.
+ * queries and keys (bf16), two fp32 values per query row, and fp32 sums of the
+ * key and value gradients (64 floats each per token and kv head), plus
+ * alignment. Returns 0 for invalid sizes.
  */
 size_t gptoss_attn_prefill_backward_workspace_bytes(int batch, int seqlen);
 
@@ -180,7 +181,9 @@ size_t gptoss_attn_prefill_backward_workspace_bytes(int batch, int seqlen);
  *   dout   bf16 [batch][seqlen][64][64]
  *   dq     bf16 [batch][seqlen][64][64];  dk, dv  bf16 [batch][seqlen][8][64]
  *   dsinks fp32 [64] (overwritten; accumulated with atomics, so the order of
- *          the fp32 additions varies from run to run)
+ *          the fp32 additions varies from run to run; so does that of dk and
+ *          dv, whose fp32 partial sums over chunks of queries are added in the
+ *          workspace before the final rounding to bf16)
  *   workspace of gptoss_attn_prefill_backward_workspace_bytes() bytes.
  * Products run on the tensor cores in bf16 with fp32 accumulation: the
  * rotated q, k and the probabilities and dS are rounded to bf16 first. All

@@ -235,7 +235,8 @@ def test_training_entry_points_argument_errors(lib):
         return (x + 255) // 256 * 256
     B, S = 2, 100
     rows = B * S * 64
-    assert wb(B, S) == r256(rows * 64 * 2) + r256(B * S * 8 * 64 * 2) + 2 * r256((rows + 128) * 4)
+    assert wb(B, S) == (r256(rows * 64 * 2) + r256(B * S * 8 * 64 * 2) + 2 * r256((rows + 128) * 4)
+                        + 2 * r256(B * S * 8 * 64 * 4))
     fb = lib.gptoss_attn_prefill_backward
     fb.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, sz, vp]
     ok = dict(q=16, k=32, v=48, s=64, p=80, w=0, o=96, lse=112, do=128, dq=144, dk=160,
