@@ -670,8 +670,9 @@ def run_long(args, name: str):
     slid_ms = float(seg[slid].sum()) / len(slid)
     full_tf = prefill_flops(B, S, 0) / (full_ms * 1e-3) / 1e12
     slid_tf = prefill_flops(B, S, 128) / (slid_ms * 1e-3) / 1e12
-    # algorithmic bytes of a sliding layer incl. the key pre-pass (read k, write rotated k)
-    slid_bytes = prefill_bytes(B, S) + 2.0 * B * S * NKV * D * 2
+    # algorithmic bytes of a sliding layer (q, out, k, v once each; the key
+    # pre-pass's extra read and write of k is a cost of the implementation)
+    slid_bytes = prefill_bytes(B, S)
     hbm, tf_burst, tf_sus, peak_src = load_peaks()
 
     # end to end through host buffers, one full-causal layer
