@@ -36,8 +36,12 @@
 //     dk = R(pos)^T dK' and dv as bf16 itself.
 //   bwd_dkv_finish_kernel (split tiles only): dk = R(pos)^T dK' and dv from the
 //     sums, as bf16.
-// Each CTA takes 256 tensor-memory columns and ~100 KB of shared memory, so
-// two CTAs share an SM and one's elementwise work overlaps the other's MMAs.
+// In both kernels the elementwise warps release S and dP (S^T, dP^T) as soon
+// as they have loaded them and write their bf16 results (dS; P^T and dS^T)
+// into separate double-buffered columns, so the MMAs of the next step run
+// while the elementwise work of this one finishes. A dQ CTA takes 256
+// tensor-memory columns and ~100 KB of shared memory (two CTAs per SM); a
+// dK/dV CTA takes all 512 columns (one CTA per SM).
 // Roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
 // warps 2-5 the elementwise warpgroup (thread = TMEM lane; warp w reads lanes
 // 32 (w % 4) .. 32 (w % 4) + 31).
@@ -57,7 +61,7 @@ constexpr int kTok = 16;      // query tokens per 128-row dQ tile
 constexpr int kKeys = 128;    // keys per dK/dV tile
 constexpr int kQKeys = 64;    // keys per step of the dQ kernel
 constexpr int kKTok = 8;      // query tokens (64 rows) per step of the dK/dV kernel
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr uint32_t kTile = 128 * 128;  // 128 rows of 64 bf16
 constexpr uint32_t kHalf = 64 * 128;   // 64 rows of 64 bf16
 constexpr uint32_t kTmemCols = 256;
@@ -66,6 +70,16 @@ constexpr float kScaleLog2 = 0.125f * kLog2e;
 constexpr float kScale = 0.125f;
 // TMEM columns: S (or S^T) [0,64), dP (dP^T) [64,128), dQ or dV [128,192), dK [192,256).
 constexpr uint32_t kColS = 0, kColP = 64, kColA = 128, kColB = 192;
+// dQ kernel: dS of alternate tiles in two 32-column buffers, so the next
+// tile's S and dP may overwrite theirs as soon as the elementwise warps have
+// loaded them; dQ accumulates at kColQ.
+constexpr uint32_t kColDS = 128, kColQ = 192;
+// dK/dV kernel (one CTA per SM, all 512 columns): S^T and dP^T at 0 and 64, then
+// two buffers of (P^T, dS^T) as bf16 (32 columns each), dV at 256, dK at 320.
+constexpr uint32_t kKTmemCols = 512;
+constexpr uint32_t kColPD = 128, kColDV = 256, kColDK = 320;
+// one CTA per SM: a shared-memory request above half of the SM's
+constexpr uint32_t kDkvSmemBytes = 120 * 1024;
 
 // dq kernel shared memory
 constexpr uint32_t kQOffQ = 0, kQOffDO = kTile, kQOffK = 2 * kTile;
@@ -88,6 +102,8 @@ enum : int {
   BAR_E_DONE = BAR_S_FULL + 1,           // elementwise results in TMEM, S/dP read
   BAR_ACC_FULL = BAR_E_DONE + 1,         // the item's accumulators complete
   BAR_MMA_DONE = BAR_ACC_FULL + 1,
+  BAR_SP_FREE = BAR_MMA_DONE + 1,        // dQ kernel: S and dP loaded by the elementwise warps
+  BAR_DS_FREE = BAR_SP_FREE + 1,         // [2] dQ kernel: dS buffer read by its dQ MMAs
   NUM_BARS = BAR_MMA_DONE + 1
 };
 
@@ -106,7 +122,8 @@ struct Ctx {
 
 // Common prologue: barriers, abort flag (a timeout left in the error word
 // skips the work), tensor memory. Returns the TMEM base address.
-__device__ uint32_t setup(Ctx& ctx, uint8_t* smem, uint32_t obar, int* err) {
+__device__ uint32_t setup(Ctx& ctx, uint8_t* smem, uint32_t obar, int* err,
+                          uint32_t ncols = kTmemCols) {
   ctx.sbase = smem_u32(smem);
   ctx.obar = obar;
   ctx.abort_flag = reinterpret_cast<volatile int*>(smem + obar + NUM_BARS * 8 + 4);
@@ -123,11 +140,14 @@ __device__ uint32_t setup(Ctx& ctx, uint8_t* smem, uint32_t obar, int* err) {
     mbar_init(ctx.bar(BAR_E_DONE), 4);
     mbar_init(ctx.bar(BAR_ACC_FULL), 1);
     mbar_init(ctx.bar(BAR_MMA_DONE), 1);
+    mbar_init(ctx.bar(BAR_SP_FREE), 4);
+    mbar_init(ctx.bar(BAR_DS_FREE), 1);
+    mbar_init(ctx.bar(BAR_DS_FREE + 1), 1);
     *ctx.abort_flag = (*reinterpret_cast<volatile int*>(err) & kErrTimeout) ? 1 : 0;
     fence_barrier_init();
   }
   if ((threadIdx.x >> 5) == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_alloc(smem_u32(tmem_slot), ncols);
     tmem_relinquish();
   }
   tc_fence_before_sync();
@@ -136,12 +156,12 @@ __device__ uint32_t setup(Ctx& ctx, uint8_t* smem, uint32_t obar, int* err) {
   return *tmem_slot;
 }
 
-__device__ void teardown(uint32_t tmem) {
+__device__ void teardown(uint32_t tmem, uint32_t ncols = kTmemCols) {
   tc_fence_before_sync();
   __syncthreads();
   if ((threadIdx.x >> 5) == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, ncols);
   }
 }
 
@@ -306,30 +326,31 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
     }
   } else if (warp == 1) {
     if (lane == 0 && !skip) {
+      // S(j) and dP(j) go out as soon as the elementwise warps have loaded
+      // S(j-1) and dP(j-1); dQ += dS(j-1) K(j-1) once dS(j-1) is written (into
+      // its own columns), so the tensor core works on tile j while the
+      // elementwise warps finish tile j-1.
       bool ok = ctx.wait(BAR_Q_FULL, 0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kStages;
-        if (!(ok = ctx.wait(BAR_KV_FULL + s, (j / kStages) & 1))) break;
-        // the elementwise warps have read S and dP of the previous tile (and
-        // dQ of that tile, issued before, reads dS first: one thread's MMAs
-        // run in order)
-        if (j > 0 && !(ok = ctx.wait(BAR_E_DONE, (j - 1) & 1))) break;
-        tc_fence_after_sync();
-        if (j > 0) {
-          const int sp = (j - 1) % kStages;
-          mma_tmem_a(tmem + kColA, tmem + kColS, ctx.sbase + kQOffK + sp * kHalf, j > 1);
-          mma_commit(ctx.bar(BAR_KV_EMPTY + sp));
+      for (int j = 0; ok && j <= n_tiles; ++j) {
+        if (j < n_tiles) {
+          const int s = j % kStages;
+          if (!(ok = ctx.wait(BAR_KV_FULL + s, (j / kStages) & 1))) break;
+          if (j > 0 && !(ok = ctx.wait(BAR_SP_FREE, (j - 1) & 1))) break;
+          tc_fence_after_sync();
+          mma_abt(tmem + kColS, ctx.sbase + kQOffQ, ctx.sbase + kQOffK + s * kHalf);
+          mma_abt(tmem + kColP, ctx.sbase + kQOffDO, ctx.sbase + kQOffV + s * kHalf);
+          mma_commit(ctx.bar(BAR_S_FULL));
         }
-        mma_abt(tmem + kColS, ctx.sbase + kQOffQ, ctx.sbase + kQOffK + s * kHalf);
-        mma_abt(tmem + kColP, ctx.sbase + kQOffDO, ctx.sbase + kQOffV + s * kHalf);
-        mma_commit(ctx.bar(BAR_S_FULL));
-      }
-      if (ok && (ok = ctx.wait(BAR_E_DONE, (n_tiles - 1) & 1))) {
-        tc_fence_after_sync();
-        const int sp = (n_tiles - 1) % kStages;
-        mma_tmem_a(tmem + kColA, tmem + kColS, ctx.sbase + kQOffK + sp * kHalf, n_tiles > 1);
-        mma_commit(ctx.bar(BAR_KV_EMPTY + sp));
-        mma_commit(ctx.bar(BAR_ACC_FULL));
+        if (j > 0) {
+          const int jp = j - 1, sp = jp % kStages;
+          if (!(ok = ctx.wait(BAR_E_DONE, jp & 1))) break;
+          tc_fence_after_sync();
+          mma_tmem_a(tmem + kColQ, tmem + kColDS + 32 * (jp & 1), ctx.sbase + kQOffK + sp * kHalf,
+                     jp > 0);
+          mma_commit(ctx.bar(BAR_KV_EMPTY + sp));
+          mma_commit(ctx.bar(BAR_DS_FREE + (jp & 1)));
+          if (jp == n_tiles - 1) mma_commit(ctx.bar(BAR_ACC_FULL));
+        }
       }
       mma_commit(ctx.bar(BAR_MMA_DONE));
       volatile int never = 0;
@@ -354,25 +375,38 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
       const int kb = (jt0 + j) * kQKeys;
       const int c_hi = t - kb;                           // visible columns [c_lo, c_hi]
       const int c_lo = W > 0 ? t - W + 1 - kb : -1;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t sv[32], pv[32], out[16];
-        tmem_ld32(tmem + lane_off + kColS + 32 * c, sv);
-        tmem_ld32(tmem + lane_off + kColP + 32 * c, pv);
+      uint32_t sv[64], pv[64], out[32];
+      tmem_ld32(tmem + lane_off + kColS, *reinterpret_cast<uint32_t(*)[32]>(sv));
+      tmem_ld32(tmem + lane_off + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+      tmem_ld32(tmem + lane_off + kColP, *reinterpret_cast<uint32_t(*)[32]>(pv));
+      tmem_ld32(tmem + lane_off + kColP + 32, *reinterpret_cast<uint32_t(*)[32]>(pv + 32));
+      // S and dP are in registers: the next tile's may overwrite them
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ctx.bar(BAR_SP_FREE));
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float ds[2];
+      for (int e = 0; e < 64; e += 2) {
+        float ds[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = 32 * c + e + u;
-            const bool vis = row_ok && col <= c_hi && col >= c_lo;
-            const float p = vis ? ex2_approx(__uint_as_float(sv[e + u]) * kScaleLog2 - lse2) : 0.f;
-            ds[u] = p * (__uint_as_float(pv[e + u]) - dd) * kScale;
-          }
-          out[e / 2] = pack_bf16x2(ds[0], ds[1]);
+        for (int u = 0; u < 2; ++u) {
+          const int col = e + u;
+          const bool vis = row_ok && col <= c_hi && col >= c_lo;
+          const float p = vis ? ex2_approx(__uint_as_float(sv[e + u]) * kScaleLog2 - lse2) : 0.f;
+          ds[u] = p * (__uint_as_float(pv[e + u]) - dd) * kScale;
         }
-        // dS (bf16 pairs) into S's columns [16c, 16c+16), all of which were read already
-        tmem_st16(tmem + lane_off + kColS + 16 * c, out);
+        out[e / 2] = pack_bf16x2(ds[0], ds[1]);
+      }
+      // this tile's dS buffer was last read by dQ of tile j-2
+      if (j >= 2 && !(ok = ctx.wait_warp(BAR_DS_FREE + (j & 1), ((j >> 1) - 1) & 1))) break;
+      tc_fence_after_sync();
+      {
+        uint32_t o16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o16[i] = out[i];
+        tmem_st16(tmem + lane_off + kColDS + 32 * (j & 1), o16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o16[i] = out[16 + i];
+        tmem_st16(tmem + lane_off + kColDS + 32 * (j & 1) + 16, o16);
       }
       tmem_st_wait();
       tc_fence_before_sync();
@@ -382,8 +416,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
     if (ok && (ok = ctx.wait_warp(BAR_ACC_FULL, 0))) {
       tc_fence_after_sync();
       uint32_t lo[32], hi[32];
-      tmem_ld32(tmem + lane_off + kColA, lo);
-      tmem_ld32(tmem + lane_off + kColA + 32, hi);
+      tmem_ld32(tmem + lane_off + kColQ, lo);
+      tmem_ld32(tmem + lane_off + kColQ + 32, hi);
       if (row_ok) {
         const int p = bwd::clamp_pos(__ldg(a.pos + static_cast<int64_t>(b) * S + t), a.err);
         unrotate_store(lo, hi, a.rope + static_cast<size_t>(p) * kRopePairs,
@@ -396,7 +430,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
 }
 
 // Partial dK and dV for one (b, g, 128-key tile, chunk of query steps) per CTA.
-__global__ void __launch_bounds__(bwd::kThreads, 2)
+__global__ void __launch_bounds__(bwd::kThreads, 1)
     bwd_dkv_kernel(const __grid_constant__ BackwardMaps maps, const BackwardArgs a) {
   using namespace bwd;
   const int S = a.seqlen, W = a.window;
@@ -418,7 +452,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   Ctx ctx;
-  const uint32_t tmem = setup(ctx, smem, kKOffBar, a.err);
+  const uint32_t tmem = setup(ctx, smem, kKOffBar, a.err, kKTmemCols);
   const bool skip = *ctx.abort_flag != 0;
   const int warp = static_cast<int>(threadIdx.x >> 5), lane = static_cast<int>(threadIdx.x & 31);
   const float* lse2_g = a.lse2 + (static_cast<int64_t>(b) * kNumKvHeads + g) * S * kGroup;
@@ -459,32 +493,33 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
     }
   } else if (warp == 1) {
     if (lane == 0 && !skip) {
+      // S^T(j), dP^T(j) go out as soon as the elementwise warps have loaded
+      // step j-1's; dV, dK of step j-1 once its P^T and dS^T are written (into
+      // buffer (j-1) & 1), so the tensor core works on step j meanwhile.
       bool ok = ctx.wait(BAR_KV_FULL, 0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kStages;
-        if (!(ok = ctx.wait(BAR_Q_FULL + s, (j / kStages) & 1))) break;
-        if (j > 0 && !(ok = ctx.wait(BAR_E_DONE, (j - 1) & 1))) break;
-        tc_fence_after_sync();
-        if (j > 0) {
-          const int sp = (j - 1) % kStages;
-          const uint32_t st = ctx.sbase + kKOffQ + sp * 2 * kHalf;
-          mma_tmem_a(tmem + kColA, tmem + kColS, st + kHalf, j > 1);  // dV += P^T dO
-          mma_tmem_a(tmem + kColB, tmem + kColP, st, j > 1);          // dK += dS^T Q'
-          mma_commit(ctx.bar(BAR_Q_EMPTY + sp));
+      for (int j = 0; ok && j <= n_tiles; ++j) {
+        if (j < n_tiles) {
+          const int s = j % kStages;
+          if (!(ok = ctx.wait(BAR_Q_FULL + s, (j / kStages) & 1))) break;
+          if (j > 0 && !(ok = ctx.wait(BAR_SP_FREE, (j - 1) & 1))) break;
+          tc_fence_after_sync();
+          const uint32_t st = ctx.sbase + kKOffQ + s * 2 * kHalf;
+          mma_abt(tmem + kColS, ctx.sbase + kKOffK, st);          // S^T = K' Q'^T
+          mma_abt(tmem + kColP, ctx.sbase + kKOffV, st + kHalf);  // dP^T = V dO^T
+          mma_commit(ctx.bar(BAR_S_FULL));
         }
-        const uint32_t st = ctx.sbase + kKOffQ + s * 2 * kHalf;
-        mma_abt(tmem + kColS, ctx.sbase + kKOffK, st);           // S^T = K' Q'^T
-        mma_abt(tmem + kColP, ctx.sbase + kKOffV, st + kHalf);   // dP^T = V dO^T
-        mma_commit(ctx.bar(BAR_S_FULL));
-      }
-      if (ok && (ok = ctx.wait(BAR_E_DONE, (n_tiles - 1) & 1))) {
-        tc_fence_after_sync();
-        const int sp = (n_tiles - 1) % kStages;
-        const uint32_t st = ctx.sbase + kKOffQ + sp * 2 * kHalf;
-        mma_tmem_a(tmem + kColA, tmem + kColS, st + kHalf, n_tiles > 1);
-        mma_tmem_a(tmem + kColB, tmem + kColP, st, n_tiles > 1);
-        mma_commit(ctx.bar(BAR_Q_EMPTY + sp));
-        mma_commit(ctx.bar(BAR_ACC_FULL));
+        if (j > 0) {
+          const int jp = j - 1, sp = jp % kStages;
+          if (!(ok = ctx.wait(BAR_E_DONE, jp & 1))) break;
+          tc_fence_after_sync();
+          const uint32_t st = ctx.sbase + kKOffQ + sp * 2 * kHalf;
+          const uint32_t pd = tmem + kColPD + 64 * (jp & 1);
+          mma_tmem_a(tmem + kColDV, pd, st + kHalf, jp > 0);  // dV += P^T dO
+          mma_tmem_a(tmem + kColDK, pd + 32, st, jp > 0);     // dK += dS^T Q'
+          mma_commit(ctx.bar(BAR_Q_EMPTY + sp));
+          mma_commit(ctx.bar(BAR_DS_FREE + (jp & 1)));
+          if (jp == n_tiles - 1) mma_commit(ctx.bar(BAR_ACC_FULL));
+        }
       }
       mma_commit(ctx.bar(BAR_MMA_DONE));
       volatile int never = 0;
@@ -505,28 +540,45 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
       // column col is token t0 + col/8: visible iff kj <= t < S and t < kj + W
       const int lo_t = kj - t0;                              // first visible token offset
       const int hi_t = min(S - 1 - t0, W > 0 ? kj + W - 1 - t0 : 1 << 30);
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t sv[32], pv[32], pw[16], dw[16];
-        tmem_ld32(tmem + lane_off + kColS + 32 * c, sv);
-        tmem_ld32(tmem + lane_off + kColP + 32 * c, pv);
+      uint32_t sv[64], pv[64], pw[32], dw[32];
+      tmem_ld32(tmem + lane_off + kColS, *reinterpret_cast<uint32_t(*)[32]>(sv));
+      tmem_ld32(tmem + lane_off + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+      tmem_ld32(tmem + lane_off + kColP, *reinterpret_cast<uint32_t(*)[32]>(pv));
+      tmem_ld32(tmem + lane_off + kColP + 32, *reinterpret_cast<uint32_t(*)[32]>(pv + 32));
+      // S^T and dP^T are in registers: the next step's may overwrite them
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ctx.bar(BAR_SP_FREE));
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float p[2], ds[2];
+      for (int e = 0; e < 64; e += 2) {
+        float p[2], ds[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = 32 * c + e + u;
-            const int tt = col >> 3;
-            const bool vis = tt >= lo_t && tt <= hi_t;
-            p[u] = vis ? ex2_approx(__uint_as_float(sv[e + u]) * kScaleLog2 - ld[col]) : 0.f;
-            // rows past the sequence carry no lse or D: keep them out of dK
-            ds[u] = vis ? p[u] * (__uint_as_float(pv[e + u]) - ld[64 + col]) * kScale : 0.f;
-          }
-          pw[e / 2] = pack_bf16x2(p[0], p[1]);
-          dw[e / 2] = pack_bf16x2(ds[0], ds[1]);
+        for (int u = 0; u < 2; ++u) {
+          const int col = e + u;
+          const int tt = col >> 3;
+          const bool vis = tt >= lo_t && tt <= hi_t;
+          p[u] = vis ? ex2_approx(__uint_as_float(sv[e + u]) * kScaleLog2 - ld[col]) : 0.f;
+          // rows past the sequence carry no lse or D: keep them out of dK
+          ds[u] = vis ? p[u] * (__uint_as_float(pv[e + u]) - ld[64 + col]) * kScale : 0.f;
         }
-        tmem_st16(tmem + lane_off + kColS + 16 * c, pw);
-        tmem_st16(tmem + lane_off + kColP + 16 * c, dw);
+        pw[e / 2] = pack_bf16x2(p[0], p[1]);
+        dw[e / 2] = pack_bf16x2(ds[0], ds[1]);
+      }
+      // this step's P^T/dS^T buffer was last read by dV, dK of step j-2
+      if (j >= 2 && !(ok = ctx.wait_warp(BAR_DS_FREE + (j & 1), ((j >> 1) - 1) & 1))) break;
+      tc_fence_after_sync();
+      {
+        const uint32_t pd = tmem + lane_off + kColPD + 64 * (j & 1);
+        uint32_t t16[16];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) t16[i] = pw[16 * h + i];
+          tmem_st16(pd + 16 * h, t16);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) t16[i] = dw[16 * h + i];
+          tmem_st16(pd + 32 + 16 * h, t16);
+        }
       }
       tmem_st_wait();
       tc_fence_before_sync();
@@ -537,8 +589,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
       tc_fence_after_sync();
       uint32_t lo[32], hi[32];
       const int64_t row = ((static_cast<int64_t>(b) * S + kj) * kNumKvHeads + g) * kHeadDim;
-      tmem_ld32(tmem + lane_off + kColA, lo);
-      tmem_ld32(tmem + lane_off + kColA + 32, hi);
+      tmem_ld32(tmem + lane_off + kColDV, lo);
+      tmem_ld32(tmem + lane_off + kColDV + 32, hi);
       if (kj < S) {
         if (a.kv_chunks > 1) {
           red_add_row(a.dv32 + row, lo, hi);
@@ -560,8 +612,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
           }
         }
       }
-      tmem_ld32(tmem + lane_off + kColB, lo);
-      tmem_ld32(tmem + lane_off + kColB + 32, hi);
+      tmem_ld32(tmem + lane_off + kColDK, lo);
+      tmem_ld32(tmem + lane_off + kColDK + 32, hi);
       if (kj < S) {
         if (a.kv_chunks > 1) {
           red_add_row(a.dk32 + row, lo, hi);
@@ -572,7 +624,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 2)
       }
     }
   }
-  teardown(tmem);
+  teardown(tmem, kKTmemCols);
 }
 
 // dk = R(pos)^T dK' and dv from the fp32 sums, as bf16: one thread per
@@ -650,7 +702,7 @@ cudaError_t launch_backward(const BackwardMaps& maps, const BackwardArgs& args, 
                            static_cast<int>(bwd::kSmemBytes));
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(bwd::kSmemBytes));
+                           static_cast<int>(bwd::kDkvSmemBytes));
   if (e != cudaSuccess) return e;
   const unsigned n_dq = static_cast<unsigned>(args.n_qt * kNumKvHeads * args.batch);
   bwd_dq_kernel<<<n_dq, bwd::kThreads, bwd::kSmemBytes, stream>>>(maps, args);
@@ -664,7 +716,7 @@ cudaError_t launch_backward(const BackwardMaps& maps, const BackwardArgs& args, 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_dkv);
   cfg.blockDim = dim3(bwd::kThreads);
-  cfg.dynamicSmemBytes = bwd::kSmemBytes;
+  cfg.dynamicSmemBytes = bwd::kDkvSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
