@@ -1,5 +1,6 @@
 // C-ABI entry points of libgptoss_attn.so: argument validation, per-device
-// state (rotary table, error word), TMA tensor maps, kernel launches.
+// state (rotary tables, per-stream error words), TMA tensor maps, kernel
+// launches.
 #include <cstdint>
 #include <mutex>
 
@@ -12,9 +13,14 @@ namespace {
 using namespace gqa;
 
 constexpr int kMaxDevices = 64;
+// Error words per device: one per stream that has launched work, in order of
+// first use; streams beyond the last word share it.
+constexpr int kErrWords = 64;
 
 struct DeviceState {
-  int* err = nullptr;         // 4-byte error word
+  int* err = nullptr;                       // kErrWords 4-byte error words
+  cudaStream_t err_stream[kErrWords] = {};  // the stream each word belongs to
+  int err_used = 0;
   float2* rope = nullptr;     // [kMaxPosition][32], plain RoPE
   float2* yarn = nullptr;     // [kMaxPosition][32], YaRN (built on first use)
   int num_sms = 0;
@@ -49,7 +55,7 @@ int build_table(float2** dst, bool yarn) {
   return GPTOSS_ATTN_OK;
 }
 
-// Allocates the error word (and, when asked, builds a rotary table) once
+// Allocates the error words (and, when asked, builds a rotary table) once
 // per device. Runs on the legacy default stream and waits for completion.
 int ensure_state(int dev, Rope need) {
   std::lock_guard<std::mutex> lock(g_mutex);
@@ -59,8 +65,9 @@ int ensure_state(int dev, Rope need) {
     return GPTOSS_ATTN_ERR_NO_DEVICE;
   if (!st.err) {
     int* e = nullptr;
-    if (cudaMalloc(&e, sizeof(int)) != cudaSuccess) return GPTOSS_ATTN_ERR_ALLOC;
-    if (cudaMemset(e, 0, sizeof(int)) != cudaSuccess) {
+    if (cudaMalloc(&e, sizeof(int) * kErrWords) != cudaSuccess) return GPTOSS_ATTN_ERR_ALLOC;
+    if (cudaMemset(e, 0, sizeof(int) * kErrWords) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess) {
       cudaFree(e);
       return GPTOSS_ATTN_ERR_LAUNCH;
     }
@@ -69,6 +76,21 @@ int ensure_state(int dev, Rope need) {
   if (need == Rope::kPlain && !st.rope) return build_table(&st.rope, false);
   if (need == Rope::kYarn && !st.yarn) return build_table(&st.yarn, true);
   return GPTOSS_ATTN_OK;
+}
+
+// The error word of `stream` on device `dev` (its state already allocated):
+// kernels launched on the stream report into it and skip their work while it
+// holds a timeout; gptoss_attn_check(stream) reads and clears it.
+int* err_word(int dev, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& st = g_state[dev];
+  for (int i = 0; i < st.err_used; ++i)
+    if (st.err_stream[i] == stream) return st.err + i;
+  if (st.err_used < kErrWords) {
+    st.err_stream[st.err_used] = stream;
+    return st.err + st.err_used++;
+  }
+  return st.err + (kErrWords - 1);
 }
 
 const float2* table_of(int dev, Rope r) {
@@ -176,7 +198,7 @@ static int prefill_impl(const void* q, const void* k, const void* v, const float
   args.pos = pos;
   args.sinks = sinks;
   args.rope = table_of(dev, rope);
-  args.err = g_state[dev].err;
+  args.err = err_word(dev, stream);
   args.out = out;
   args.lse = lse;
   args.batch = batch;
@@ -239,7 +261,7 @@ static int prefill_chunk_impl(const void* q, const void* k, const void* v, const
   args.pos = pos;
   args.sinks = sinks;
   args.rope = table_of(dev, rope);
-  args.err = g_state[dev].err;
+  args.err = err_word(dev, stream);
   args.out = out;
   args.lse = nullptr;
   args.batch = batch;
@@ -315,7 +337,7 @@ static int decode_impl(const void* q, const void* kcache, const void* vcache, co
   const size_t rows = static_cast<size_t>(batch) * kNumHeads * nsplit;
   a.part_o = static_cast<float*>(workspace);
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + rows * kHeadDim * 4);
-  a.err = g_state[dev].err;
+  a.err = err_word(dev, stream);
   a.batch = batch;
   a.max_len = max_len;
   a.window = window > 0 ? window : 0;
@@ -450,7 +472,7 @@ int gptoss_attn_prefill_backward(const void* q, const void* k, const void* v, co
   a.pos = pos;
   a.sinks = sinks;
   a.rope = table_of(dev, Rope::kPlain);
-  a.err = g_state[dev].err;
+  a.err = err_word(dev, stream);
   a.lse = lse;
   a.out = static_cast<const uint16_t*>(out);
   a.dout = static_cast<const uint16_t*>(dout);
@@ -491,7 +513,7 @@ int gptoss_attn_debug_wait_timeout(unsigned timeout_us, cudaStream_t stream) {
   int st = current_device(&dev);
   if (st == GPTOSS_ATTN_OK) st = ensure_state(dev, Rope::kNone);
   if (st != GPTOSS_ATTN_OK) return st;
-  return launch_wait_timeout(g_state[dev].err, static_cast<uint64_t>(timeout_us) * 1000u,
+  return launch_wait_timeout(err_word(dev, stream), static_cast<uint64_t>(timeout_us) * 1000u,
                              stream) == cudaSuccess
              ? GPTOSS_ATTN_OK
              : GPTOSS_ATTN_ERR_LAUNCH;
@@ -502,15 +524,18 @@ int gptoss_attn_check(cudaStream_t stream) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return GPTOSS_ATTN_ERR_NO_DEVICE;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return GPTOSS_ATTN_ERR_LAUNCH;
-  int* e = nullptr;
+  bool allocated = false;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    e = g_state[dev].err;
+    allocated = g_state[dev].err != nullptr;
   }
-  if (!e) return GPTOSS_ATTN_OK;
+  if (!allocated) return GPTOSS_ATTN_OK;
+  int* e = err_word(dev, stream);
+  // Only this stream is waited on: the word is this stream's alone.
   int h = 0;
-  if (cudaMemcpy(&h, e, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
-      cudaMemset(e, 0, sizeof(int)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+  if (cudaMemcpyAsync(&h, e, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaMemsetAsync(e, 0, sizeof(int), stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
     return GPTOSS_ATTN_ERR_LAUNCH;
   if (h & kErrTimeout) return GPTOSS_ATTN_ERR_DEVICE_TIMEOUT;
   if (h & kErrPosition) return GPTOSS_ATTN_ERR_BAD_POSITION;

@@ -31,8 +31,10 @@
  *   - Calls are asynchronous on `stream` (0 = legacy default stream).
  *   - The return value is GPTOSS_ATTN_OK (0) or a negative status code;
  *     no call aborts or prints. Argument errors are reported before any
- *     work is enqueued. Faults detected inside a kernel set a device error
- *     word that gptoss_attn_check() reports and clears.
+ *     work is enqueued. Faults detected inside a kernel set the error word
+ *     of the stream it was launched on, which gptoss_attn_check(stream)
+ *     reports and clears. Each device keeps 64 such words, given to streams
+ *     in order of first use; streams beyond the 64th share the last word.
  *   - Accumulation is fp32; the rotated q/k and the probabilities are
  *     rounded to bf16 for the tensor-core products; the output is rounded
  *     to bf16 once.
@@ -297,7 +299,7 @@ int gptoss_attn_decode_yarn(const void* q, const void* kcache, const void* vcach
  * them on one stream or otherwise serialize them. Device-side conditions of
  * this path (a length outside [0, max_len], which is clamped; a pipeline
  * timeout) are not reported by gptoss_attn_check(), and this path keeps
- * running while the device error word of the other entry points holds a
+ * running while the stream's error word of the other entry points holds a
  * timeout.
  */
 #define GPTOSS_ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
@@ -311,19 +313,21 @@ int gptoss_attn_decode_noalloc(const void* q, const void* kcache, const void* vc
  * path every kernel pipeline wait uses. One thread waits, through the same
  * bounded wait, on a barrier that nothing arrives at; after timeout_us
  * microseconds (1 .. 2000000, else GPTOSS_ATTN_ERR_BAD_SHAPE) the wait gives
- * up, sets the timeout bit of the device error word and the kernel returns, so
- * the context stays usable. Until gptoss_attn_check() clears the word,
- * prefill and decode kernels launched on this device skip their work; check
- * then reports GPTOSS_ATTN_ERR_DEVICE_TIMEOUT. Asynchronous on `stream`.
+ * up, sets the timeout bit of `stream`'s error word and the kernel returns, so
+ * the context stays usable. Until gptoss_attn_check(stream) clears the word,
+ * prefill, decode and backward kernels launched on `stream` skip their work
+ * (other streams are not affected); check then reports
+ * GPTOSS_ATTN_ERR_DEVICE_TIMEOUT. Asynchronous on `stream`.
  */
 int gptoss_attn_debug_wait_timeout(unsigned timeout_us, cudaStream_t stream);
 
 /*
- * Synchronizes `stream`, then reads and clears the current device's error
- * word. Returns GPTOSS_ATTN_OK, GPTOSS_ATTN_ERR_DEVICE_TIMEOUT,
- * GPTOSS_ATTN_ERR_BAD_POSITION, GPTOSS_ATTN_ERR_BAD_LENGTH or
- * GPTOSS_ATTN_ERR_LAUNCH (a CUDA error surfaced by the synchronization).
- * While the error word is set, kernels skip their work.
+ * Synchronizes `stream`, then reads and clears its error word on the current
+ * device (stream-ordered; no other stream is waited on). Returns
+ * GPTOSS_ATTN_OK, GPTOSS_ATTN_ERR_DEVICE_TIMEOUT, GPTOSS_ATTN_ERR_BAD_POSITION,
+ * GPTOSS_ATTN_ERR_BAD_LENGTH or GPTOSS_ATTN_ERR_LAUNCH (a CUDA error surfaced
+ * by the synchronization). While a stream's word holds a timeout, kernels
+ * launched on that stream skip their work.
  */
 int gptoss_attn_check(cudaStream_t stream);
 

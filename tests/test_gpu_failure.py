@@ -97,3 +97,28 @@ def test_backward_skips_work_while_a_timeout_is_pending(cuda_device):
     gqa.check()
     for g, r in zip(grads[:3], ref[:3]):
         assert torch.equal(g, r)
+
+
+@pytest.mark.gpu
+def test_timeout_stays_on_its_stream(cuda_device):
+    """Error words are per stream: a timeout pending on one stream does not
+    make kernels on another stream skip their work, and only a check of its
+    own stream reports it."""
+    lib = gqa._load()
+    x = synth.make_prefill_inputs(1, 1, 1, 70)
+    q, k, v = bits_to_dev(x["q"]), bits_to_dev(x["k"]), bits_to_dev(x["v"])
+    sinks, pos = torch.from_numpy(x["sinks"]).cuda(), torch.from_numpy(x["pos"]).cuda()
+    side = torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+    gqa.check(side)
+    gqa.check(main)
+    assert lib.gptoss_attn_debug_wait_timeout(1000, side.cuda_stream) == 0
+    torch.cuda.synchronize()
+    out = torch.full((1, 70, 64, 64), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gqa.prefill(q, k, v, sinks, pos, 0, out=out, stream=main)
+    assert lib.gptoss_attn_check(main.cuda_stream) == 0
+    qf, kf, vf = (synth.bf16_bits_to_f64(x[n]) for n in ("q", "k", "v"))
+    compare(dev_to_f64(out), oracle.prefill(qf, kf, vf, x["sinks"], x["pos"], 0),
+            "prefill on another stream")
+    assert lib.gptoss_attn_check(side.cuda_stream) == DEVICE_TIMEOUT
+    assert lib.gptoss_attn_check(side.cuda_stream) == 0

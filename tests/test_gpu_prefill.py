@@ -169,13 +169,16 @@ def _sample_rows(B, S, seed, n_random=128):
 
 
 @pytest.mark.parametrize("config,B,S,layer,window", [
-    (3, 4, 16384, 0, 128), (3, 4, 16384, 1, 0),
-    (5, 1, 131072, 0, 0), (5, 1, 131072, 1, 128)])
+    (3, 4, 16384, 0, 128), (3, 4, 16384, 1, 0), (3, 4, 16384, 22, 128), (3, 4, 16384, 23, 0),
+    (5, 1, 131072, 0, 0), (5, 1, 131072, 1, 128),
+    (7, 1, 4096, 0, 128), (7, 1, 4096, 1, 0), (7, 1, 4096, 34, 128), (7, 1, 4096, 35, 0)])
 def test_full_size_sampled_rows(cuda_device, config, B, S, layer, window):
     """Full-size layers in the launch configuration the bench times, with the
     bench's inputs (the seeded recipe drawn on the device); the oracle checks
     the first and last 256 tokens, the window edge and random tokens of every
-    sequence, all 64 heads."""
+    sequence, all 64 heads. Config 3's first and last layer pairs, config 5's
+    two layers, and the first and last layer pairs of the 36-layer stack
+    (seed recipe 7, B=1 S=4096)."""
     from synth import device as sdev
     dev = torch.device("cuda")
     q = sdev.bf16_normal(synth.seed_for(config, layer, synth.TENSOR_Q), (B, S, NQ, D), dev)
