@@ -102,10 +102,12 @@ enum : int {
   BAR_E_DONE = BAR_S_FULL + 1,           // elementwise results in TMEM, S/dP read
   BAR_ACC_FULL = BAR_E_DONE + 1,         // the item's accumulators complete
   BAR_MMA_DONE = BAR_ACC_FULL + 1,
-  BAR_SP_FREE = BAR_MMA_DONE + 1,        // dQ kernel: S and dP loaded by the elementwise warps
-  BAR_DS_FREE = BAR_SP_FREE + 1,         // [2] dQ kernel: dS buffer read by its dQ MMAs
-  NUM_BARS = BAR_MMA_DONE + 1
+  BAR_SP_FREE = BAR_MMA_DONE + 1,        // S and dP (S^T and dP^T) loaded by the elementwise warps
+  BAR_DS_FREE = BAR_SP_FREE + 1,         // [2] a bf16 result buffer read by its MMAs
+  NUM_BARS = BAR_DS_FREE + 2
 };
+// the barriers, then the TMEM address slot and the abort flag (8 bytes)
+static_assert(NUM_BARS * 8 + 8 <= 256, "barrier region");
 
 struct Ctx {
   uint32_t sbase, obar;
